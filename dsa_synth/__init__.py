@@ -1,0 +1,219 @@
+"""Seeded synthetic inputs for the lightning indexer (score + top-k).
+
+This module is shared by the fp64 oracle and the CUDA path. It draws the
+inputs and encodes them into the storage formats the indexer reads (bf16 bit
+patterns; fp8-e4m3 bytes with block-32 e8m0 scale bytes). It holds none of the
+indexer's arithmetic: it never decodes a stored value back into a number and
+never computes a score or a selection.
+
+Recipe (all workloads): ``numpy.random.default_rng(seed)`` (PCG64), draws in
+the order q, k, w, positions. Gaussian values are drawn as float32 in fixed
+chunks of ``CHUNK`` elements; bf16 storage is round-to-nearest-even of those
+float32 values. w is float32 ``N(0,1) * w_scale``. positions are
+``rng.integers(lo, hi)`` (int32, hi exclusive).
+
+Workload shapes follow the pages' decode and prefill statements: DeepSeek-V3.2
+Sparse Indexer Kernel API Reference (decode step, n_tokens one per sequence,
+head_dim = 128, key cache ``[n_tokens, max_seq_len, head_dim]``), and Sparse
+Attention Indexer MX BF16Score Kernel API Reference (prefill self-scoring,
+queries == keys, head_dim == 128, block-32 e8m0 scales).
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional
+
+import numpy as np
+
+CHUNK = 1 << 22          # gaussian draws per call (fixes the stream layout)
+MX_BLOCK = 32            # e8m0 scale block along D
+E4M3_MAX = 448.0         # largest finite e4m3 magnitude
+
+MODE_POSITIONS = 0       # decode: slot s valid iff s <= positions[t]
+MODE_CAUSAL = 1          # packed prefill: slot s valid iff s <= t (sequence-local)
+DTYPE_BF16 = 0
+DTYPE_FP8 = 1
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    """One synthetic indexer problem (sizes, mask rule, value distributions)."""
+    name: str
+    mode: int                      # MODE_POSITIONS or MODE_CAUSAL
+    T: int                         # query tokens
+    H: int                         # indexer heads
+    D: int                         # head_dim
+    index_topk: int
+    dtype: int = DTYPE_BF16
+    S: int = 0                     # POSITIONS: slots per sequence cache
+    shared_cache: bool = False     # POSITIONS: one cache for every token
+    pos_lo: int = 0                # POSITIONS: positions ~ U[pos_lo, pos_hi)
+    pos_hi: int = 0
+    seqlens: tuple = ()            # CAUSAL: packed sequence lengths
+    w_scale: float = 1.0
+    seed: int = 0
+
+    @property
+    def num_seqs(self) -> int:
+        if self.mode == MODE_CAUSAL:
+            return len(self.seqlens)
+        return 1 if self.shared_cache else self.T
+
+    @property
+    def key_slots(self) -> int:
+        """Rows of the key cache buffer (slots of all sequences)."""
+        if self.mode == MODE_CAUSAL:
+            return int(sum(self.seqlens))
+        return self.S * self.num_seqs
+
+    @property
+    def k_seq_stride(self) -> int:
+        """Elements between consecutive sequences' caches (POSITIONS)."""
+        if self.mode == MODE_CAUSAL or self.shared_cache:
+            return 0
+        return self.S * self.D
+
+    def cu_seqlens(self) -> np.ndarray:
+        return np.concatenate([[0], np.cumsum(self.seqlens)]).astype(np.int32)
+
+
+# The five workloads: a tiny decode case, a decode batch, a long-context fp8
+# decode, a causal prefill and a packed ragged prefill.
+WORKLOADS = {
+    "tiny_decode": Workload("tiny_decode", MODE_POSITIONS, T=4, H=4, D=128,
+                            index_topk=64, S=1024, pos_lo=64, pos_hi=1024,
+                            w_scale=1.0 / 2.0),
+    "decode_batch": Workload("decode_batch", MODE_POSITIONS, T=16, H=64, D=128,
+                             index_topk=2048, S=32768, pos_lo=2048,
+                             pos_hi=32768, w_scale=1.0 / 8.0),
+    "long_decode_fp8": Workload("long_decode_fp8", MODE_POSITIONS, T=64, H=64,
+                                D=128, index_topk=1024, dtype=DTYPE_FP8,
+                                S=131072, pos_lo=1024, pos_hi=131072,
+                                w_scale=1.0 / 8.0),
+    "prefill_causal": Workload("prefill_causal", MODE_CAUSAL, T=8192, H=64,
+                               D=128, index_topk=2048, seqlens=(8192,),
+                               w_scale=1.0 / 8.0),
+    "ragged_prefill": Workload("ragged_prefill", MODE_CAUSAL, T=118784, H=64,
+                               D=128, index_topk=2048,
+                               seqlens=(4096, 16384, 32768, 65536),
+                               w_scale=1.0 / 8.0),
+}
+
+
+def gaussian_f32(rng: np.random.Generator, n: int) -> np.ndarray:
+    """n float32 N(0,1) draws, taken in chunks of CHUNK."""
+    out = np.empty(n, dtype=np.float32)
+    for i in range(0, n, CHUNK):
+        m = min(CHUNK, n - i)
+        out[i:i + m] = rng.standard_normal(m, dtype=np.float32)
+    return out
+
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 to bf16 (nearest, ties to even); returns uint16 bits."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    out = np.empty(u.shape, dtype=np.uint16)
+    step = 1 << 24
+    flat_u, flat_o = u.reshape(-1), out.reshape(-1)
+    for i in range(0, flat_u.size, step):
+        v = flat_u[i:i + step].astype(np.uint64)
+        v = (v + 0x7FFF + ((v >> 16) & 1)) >> 16
+        flat_o[i:i + step] = v.astype(np.uint16)
+    return out
+
+
+def f32_to_mx_e4m3(x: np.ndarray):
+    """Encode float32 values [..., D] as e4m3 bytes with block-32 e8m0 scales.
+
+    Per block of 32 along D (the MX layout the pages use for ``qr_scale_hbm``,
+    ``wq_b_scale`` and ``k_scale_cache``): the scale is the power of two 2^e
+    with the smallest e such that 448 * 2^e >= amax (amax over the block,
+    floored at 448 * 2^-127 so that e >= -127); byte = e + 127. Each element is
+    then x * 2^-e rounded to the nearest e4m3 value, ties to even (|x * 2^-e|
+    <= 448, so nothing saturates). Returns (data uint8 [..., D], scale uint8
+    [..., D/32]).
+    """
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    D = x.shape[-1]
+    assert D % MX_BLOCK == 0
+    lead = x.shape[:-1]
+    blocks = x.reshape(-1, D // MX_BLOCK, MX_BLOCK)
+    data = np.empty(blocks.shape, dtype=np.uint8)
+    scale = np.empty(blocks.shape[:2], dtype=np.uint8)
+    step = max(1, (1 << 22) // D)
+    for i in range(0, blocks.shape[0], step):
+        b = blocks[i:i + step].astype(np.float64)
+        amax = np.maximum(np.abs(b).max(axis=-1), E4M3_MAX * 2.0 ** -127)
+        m, E = np.frexp(amax)                    # amax = m * 2^E, m in [0.5, 1)
+        # 448 = 0.875 * 2^9: 448 * 2^e >= m * 2^E  <=>  e >= E - 9 + log2(m/0.875)
+        e = E.astype(np.int64) - 9 + (m > 0.875)
+        assert e.min() >= -127 and e.max() <= 127
+        scale[i:i + step] = (e + 127).astype(np.uint8)
+        y = np.ldexp(b, -e[..., None])           # exact power-of-two scaling
+        data[i:i + step] = _e4m3_rne_bytes(y)
+    return data.reshape(lead + (D,)), scale.reshape(lead + (D // MX_BLOCK,))
+
+
+def _e4m3_rne_bytes(y: np.ndarray) -> np.ndarray:
+    """Nearest-even e4m3 (bias 7, 3 mantissa bits) code of |y| <= 448."""
+    a = np.abs(y)
+    sign = np.signbit(y).astype(np.uint16) << 7
+    _, F = np.frexp(a)                           # a = m * 2^F, m in [0.5, 1)
+    unb = F.astype(np.int64) - 1                 # floor(log2 a) for a > 0
+    # subnormal range (a < 2^-6): quantum 2^-9; a carry to 8 is the code of 2^-6
+    sub = np.rint(np.ldexp(a, 9))
+    # normal range: quantum 2^(unb-3); a mantissa carry to 8 bumps the exponent
+    unb_c = np.maximum(unb, -6)
+    mant = np.rint((np.ldexp(a, -unb_c) - 1.0) * 8.0)
+    normal = ((unb_c + 7) << 3) + mant.astype(np.int64)
+    code = np.where((a == 0) | (unb < -6), sub.astype(np.int64), normal)
+    assert code.max() <= 0x7E
+    return (code.astype(np.uint16) | sign).astype(np.uint8)
+
+
+def _values(rng, n, kind):
+    if kind == "int":
+        return rng.integers(-3, 4, size=n).astype(np.float32)
+    return gaussian_f32(rng, n)
+
+
+def _encode(xf, dtype):
+    if dtype == DTYPE_BF16:
+        return f32_to_bf16_bits(xf), None
+    return f32_to_mx_e4m3(xf)
+
+
+def generate(wl: Workload, value_kind: str = "gauss",
+             seed: Optional[int] = None) -> dict:
+    """Draw one workload's inputs (host numpy arrays, storage formats).
+
+    value_kind "gauss": q, k ~ N(0,1), w ~ N(0,1) * w_scale (the pages'
+    workloads). "int": q, k uniform integers in [-3, 3], w uniform in
+    {-1, -1/2, 1/2, 1}: every product and sum of the indexer is then an exact
+    fp32 value, so a correct fp32 kernel reproduces the exact result.
+
+    Keys of the returned dict: q ([T,H,D] uint16 bf16 bits or uint8 e4m3),
+    q_scale ([T,H,D/32] uint8 or None), k ([key_slots, D]), k_scale, w
+    ([T,H] float32), positions ([T] int32, POSITIONS only), cu_seqlens
+    ([num_seqs+1] int32, CAUSAL only).
+    """
+    rng = np.random.default_rng(wl.seed if seed is None else seed)
+    T, H, D = wl.T, wl.H, wl.D
+    q, q_scale = _encode(_values(rng, T * H * D, value_kind).reshape(T, H, D),
+                         wl.dtype)
+    k, k_scale = _encode(
+        _values(rng, wl.key_slots * D, value_kind).reshape(wl.key_slots, D),
+        wl.dtype)
+    if value_kind == "int":
+        w = rng.choice(np.array([-1.0, -0.5, 0.5, 1.0], dtype=np.float32),
+                       size=T * H).reshape(T, H)
+    else:
+        w = (gaussian_f32(rng, T * H) * np.float32(wl.w_scale)).reshape(T, H)
+    out = dict(q=q, q_scale=q_scale, k=k, k_scale=k_scale, w=w,
+               positions=None, cu_seqlens=None)
+    if wl.mode == MODE_POSITIONS:
+        out["positions"] = rng.integers(wl.pos_lo, wl.pos_hi, size=T,
+                                        dtype=np.int32)
+    else:
+        out["cu_seqlens"] = wl.cu_seqlens()
+    return out

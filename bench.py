@@ -1,0 +1,537 @@
+#!/usr/bin/env python
+"""Benchmark of the lightning indexer (scores + top-k) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference]
+
+One step = one dsa_indexer_forward (score kernel + top-k kernel) over one
+batch of the workload, inputs resident in HBM. Steps are replayed from CUDA
+graphs over several copies of the inputs, rotated so that the bytes touched
+between two uses of a copy exceed twice the L2. Prints ONE JSON line (rank 0).
+
+Metric: valid query.key pairs per second (score + top-k); `roofline` gives
+the dominant kernel's achieved fraction of the measured peak, `path_roofline`
+the whole step's. `e2e` repeats the measurement through the API with pinned
+host buffers and the host<->device copies inside the timed region.
+`cpu_baseline` is the fp64 oracle on a bounded sample, on the host cores.
+Multi-GPU (torchrun): every rank runs its own copy of the workload (weak
+scaling, no collective on the data path); time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import dsa_synth as syn  # noqa: E402
+
+METRIC = "indexer query·key pairs/s (score+top-k) at 1 B200, % of roofline"
+UNIT = "pairs/s"
+DEFAULTS = {   # steps, warmup, graph length
+    "tiny_decode": (100000, 5000, 500),
+    "decode_batch": (60000, 3000, 240),
+    "long_decode_fp8": (6000, 300, 60),
+    "prefill_causal": (1500, 30, 30),
+    "ragged_prefill": (20, 3, 1),
+}
+L2_BYTES = 126 * 2**20
+
+
+# ---------------------------------------------------------------- workload math
+def valid_pairs(wl, inputs) -> int:
+    if wl.mode == syn.MODE_POSITIONS:
+        p = np.asarray(inputs["positions"], np.int64)
+        return int(np.clip(p + 1, 0, wl.S).sum())
+    return int(sum(L * (L + 1) // 2 for L in wl.seqlens))
+
+
+def score_elems(wl) -> int:
+    if wl.mode == syn.MODE_POSITIONS:
+        return wl.T * wl.S
+    return int(sum(L * L for L in wl.seqlens))
+
+
+def algorithmic(wl, inputs):
+    """(flops, score-kernel bytes, top-k bytes) per step.
+
+    Bytes: q (+scales) + w + key slots that some token may attend to (+scales)
+    + the score write; top-k: its index write. The top-k's read of the score
+    rows is an implementation cost and is not counted."""
+    pairs = valid_pairs(wl, inputs)
+    elt = 1 if wl.dtype == syn.DTYPE_FP8 else 2
+    slot_bytes = wl.D * elt + (wl.D // 32 if wl.dtype == syn.DTYPE_FP8 else 0)
+    q_bytes = wl.T * wl.H * slot_bytes
+    w_bytes = wl.T * wl.H * 4
+    if wl.mode == syn.MODE_POSITIONS:
+        p = np.clip(np.asarray(inputs["positions"], np.int64) + 1, 0, wl.S)
+        k_slots = int(p.max()) if wl.shared_cache else int(p.sum())
+    else:
+        k_slots = wl.T
+    score_bytes = q_bytes + w_bytes + k_slots * slot_bytes + score_elems(wl) * 4
+    topk_bytes = wl.T * wl.index_topk * 4
+    flops = 2.0 * wl.H * wl.D * pairs
+    return flops, score_bytes, topk_bytes
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        m = json.load(open(path))
+        return dict(hbm=float(m["hbm_gbs"]), bf16=float(m["bf16_tflops"]),
+                    bf16_sust=float(m["bf16_tflops_sustained"]), src="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, src="fallback")
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    cs = os.path.join(ROOT, "sparse_attention_lightning_tcgen05_b200", "csrc")
+    for f in sorted(os.listdir(cs)):
+        h.update(open(os.path.join(cs, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the score kernel from the committed ncu
+    summary, or None when the summary is absent or the kernel source changed
+    since it was taken."""
+    path = os.path.join(ROOT, "profiles", f"score_kernel_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    txt = open(path).read()
+    mh = re.search(r"src_hash:\s*`?([0-9a-f]+)", txt)
+    mb = re.search(r"dram_bytes_per_launch:\s*`?([0-9.eE+]+)", txt)
+    if not mh or not mb or mh.group(1) != source_hash():
+        return None
+    return float(mb.group(1))
+
+
+# ---------------------------------------------------------------- ranks
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def init_dist(world: int, backend: str):
+    if world <= 1:
+        return None
+    import torch.distributed as dist
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def barrier(dist, device=None):
+    if dist is not None:
+        if device is not None:
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(dist, value: float, device) -> float:
+    """Largest `value` over all ranks (every rank calls this, in order)."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
+              "clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id           # "GPU-<uuid>" (immune to index remapping)
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(f[1]), smax=float(f[2]),
+                                 util=float(f[4]) if f[4] not in ("", "[N/A]") else 0.0,
+                                 hw=f[5], hwt=f[6], swt=f[7], pcap=f[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        loaded = [r for r in rows if r["util"] > 0] or rows
+        reasons = set()
+        for r in loaded:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": float(np.median([r["sm"] for r in loaded])),
+                "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(loaded)}
+
+
+# ---------------------------------------------------------------- our arm
+def build_sets(wl, inputs, nsets, device):
+    from sparse_attention_lightning_tcgen05_b200.problem import DeviceProblem
+    return [DeviceProblem.from_workload(wl, inputs, device=device) for _ in range(nsets)]
+
+
+def capture(fn_list, stream):
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for fn in fn_list:
+            fn()
+    return g
+
+
+def time_graphs(graphs, reps, stream):
+    """Replay graphs[0] `reps` times then graphs[1:] once; device ms."""
+    import torch
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for _ in range(reps):
+            graphs[0].replay()
+        for g in graphs[1:]:
+            g.replay()
+        end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end)
+
+
+def step_graphs(sets, which, steps, glen, stream):
+    """Graphs that run `steps` steps in total (a main graph of `glen` steps,
+    replayed, and a remainder graph)."""
+    n = len(sets)
+    calls = {"forward": lambda p: p.forward, "score": lambda p: p.score,
+             "topk": lambda p: p.run_topk}[which]
+    glen = max(1, min(glen, steps))
+    main = capture([calls(sets[i % n]) for i in range(glen)], stream)
+    rem = steps % glen
+    extra = [capture([calls(sets[i % n]) for i in range(rem)], stream)] if rem else []
+    return [main] + extra, steps // glen
+
+
+def run_ours(args, wl, dist, rank, world, device):
+    import torch
+    from sparse_attention_lightning_tcgen05_b200 import DSA_OK
+    torch.cuda.set_device(device)
+    inputs = syn.generate(wl, seed=wl.seed + rank)
+    flops, sbytes, tbytes = algorithmic(wl, inputs)
+    pairs = valid_pairs(wl, inputs)
+    per_set = sbytes
+    nsets = 1 if per_set > 2 * L2_BYTES else int(np.ceil(2 * L2_BYTES / per_set)) + 1
+    nsets = min(nsets, 8)
+    sets = build_sets(wl, inputs, nsets, device)
+    steps, warmup = args.steps, args.warmup
+    glen = DEFAULTS.get(wl.name, (0, 0, 32))[2]
+    glen = (max(1, glen // nsets)) * nsets if glen >= nsets else glen
+    stream = torch.cuda.Stream(device=device)
+
+    # eager warm-up: sets kernel attributes, checks the device status
+    with torch.cuda.stream(stream):
+        for p in sets:
+            p.forward(stream)
+    for p in sets:
+        st = p.device_status(stream)
+        if st != DSA_OK:
+            raise RuntimeError(f"device status {st} after warm-up")
+
+    fwd, fwd_reps = step_graphs(sets, "forward", steps, glen, stream)
+    wg, wreps = step_graphs(sets, "forward", max(warmup, 1), glen, stream)
+    time_graphs(wg, wreps, stream)                          # W warm-up steps
+
+    torch.cuda.synchronize(device)
+    barrier(dist, device)
+    torch.cuda.synchronize(device)
+    uuid = str(torch.cuda.get_device_properties(device).uuid)
+    with ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid) as clk:
+        ms = time_graphs(fwd, fwd_reps, stream)             # K timed steps
+    torch.cuda.synchronize(device)
+    barrier(dist, device)
+    ms_max = max_over_ranks(dist, ms, device)
+
+    # the two kernels alone, same rotation, for the roofline
+    rsteps = max(glen, min(steps, 4 * glen))
+    sg, sreps = step_graphs(sets, "score", rsteps, glen, stream)
+    tg, treps = step_graphs(sets, "topk", rsteps, glen, stream)
+    time_graphs(sg, sreps, stream)
+    ms_score = time_graphs(sg, sreps, stream) / rsteps
+    ms_topk = time_graphs(tg, treps, stream) / rsteps
+    for p in sets:
+        st = p.device_status(stream)
+        if st != DSA_OK:
+            raise RuntimeError(f"device status {st} after timing")
+
+    e2e = run_e2e(args, wl, inputs, sets[0], pairs, stream, device, dist)
+    del fwd, wg, sg, tg
+    return dict(ms_step=ms_max / steps, ms_local=ms / steps, ms_score=ms_score,
+                ms_topk=ms_topk, flops=flops, sbytes=sbytes, tbytes=tbytes,
+                pairs=pairs, nsets=nsets, clocks=clk.summary(), e2e=e2e)
+
+
+def run_e2e(args, wl, inputs, p, pairs, stream, device, dist):
+    """Through the API with pinned host buffers: per step the inputs go
+    host->device, the forward runs, scores and top-k come back."""
+    import torch
+
+    def pinned(x):
+        if x is None:
+            return None
+        a = np.ascontiguousarray(x)
+        if a.dtype == np.uint16:
+            a = a.view(np.int16)
+        return torch.from_numpy(a).pin_memory()
+    host = {k: pinned(inputs.get(k)) for k in ("q", "q_scale", "w", "k", "k_scale",
+                                                "positions", "cu_seqlens")}
+    dev = {"q": p.q, "q_scale": p.q_scale, "w": p.w, "k": p.k_cache,
+           "k_scale": p.k_scale, "positions": p.positions, "cu_seqlens": p.cu_seqlens}
+    out_s = torch.empty(p.scores.shape, dtype=p.scores.dtype).pin_memory()
+    out_t = torch.empty(p.topk.shape, dtype=p.topk.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+    d2h = out_s.numel() * 4 + out_t.numel() * 4
+    n = args.e2e_steps
+
+    def step():
+        for k, v in host.items():
+            if v is not None:
+                dev[k].copy_(v, non_blocking=True)
+        p.forward(stream)
+        out_s.copy_(p.scores, non_blocking=True)
+        out_t.copy_(p.topk, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            step()
+        torch.cuda.synchronize(device)
+        barrier(dist, device)
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for _ in range(n):
+            step()
+        end.record(stream)
+    end.synchronize()
+    ms = max_over_ranks(dist, start.elapsed_time(end), device)
+    world = dist.get_world_size() if dist is not None else 1
+    return {"value": pairs * n * world / (ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "steps": n}
+
+
+# ---------------------------------------------------------------- the oracle
+def oracle_sample_rows(wl, inputs, pair_budget: int, start: int = 0):
+    """Query rows, taken round-robin from `start`, until the sample holds
+    about `pair_budget` valid pairs (at least one row)."""
+    if wl.mode == syn.MODE_POSITIONS:
+        nv = np.clip(np.asarray(inputs["positions"], np.int64) + 1, 0, wl.S)
+    else:
+        cu = wl.cu_seqlens().astype(np.int64)
+        nv = np.empty(wl.T, np.int64)
+        for i in range(len(wl.seqlens)):
+            nv[cu[i]:cu[i + 1]] = np.arange(1, wl.seqlens[i] + 1)
+    # spread the sample over the workload: a fixed stride through the rows
+    stride = max(1, wl.T // 64) if wl.T > 64 else 1
+    order = np.concatenate([np.arange(o, wl.T, stride) for o in range(stride)])
+    order = np.roll(order, -start)
+    rows, total = [], 0
+    for t in order:
+        rows.append(int(t))
+        total += int(nv[t])
+        if total >= pair_budget:
+            break
+    return rows, total
+
+
+def time_oracle(wl, inputs, rows, nthreads):
+    import oracle
+    P = oracle.Problem(wl, inputs)
+    t0 = time.perf_counter()
+    sc = P.scores(rows, nthreads=nthreads)
+    P.topk(rows, sc, wl.index_topk, nthreads=nthreads)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(wl, inputs, budget_s=15.0):
+    """The oracle, as it is, on a bounded sample of the workload."""
+    cores = os.cpu_count() or 1
+    rows, pairs = oracle_sample_rows(wl, inputs, 2000)
+    dt = time_oracle(wl, inputs, rows, cores)
+    rate = pairs / max(dt, 1e-9)
+    target = int(min(valid_pairs(wl, inputs), max(pairs, rate * budget_s * 0.5)))
+    rows, pairs = oracle_sample_rows(wl, inputs, target)
+    dt = time_oracle(wl, inputs, rows, cores)
+    return {"value": pairs / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{len(rows)} of {wl.T} query rows of {wl.name} ({pairs} valid "
+                      f"pairs), fp64 scores + top-k, {dt:.2f} s"}
+
+
+def run_reference(args, wl):
+    """The fp64 oracle as the reference arm: each step scores and selects a
+    bounded sample of rows, sized so that the whole run takes a few minutes."""
+    inputs = syn.generate(wl)
+    cores = os.cpu_count() or 1
+    rows, pairs = oracle_sample_rows(wl, inputs, 2000)
+    dt = time_oracle(wl, inputs, rows, cores)
+    rate = pairs / max(dt, 1e-9)
+    per_step_s = max(0.002, 150.0 / (args.steps + args.warmup))
+    budget = int(max(1, rate * per_step_s))
+    for i in range(args.warmup):
+        r, _ = oracle_sample_rows(wl, inputs, budget, start=i)
+        time_oracle(wl, inputs, r, cores)
+    total_pairs, total_s, nrows = 0, 0.0, 0
+    for i in range(args.steps):
+        r, pr = oracle_sample_rows(wl, inputs, budget, start=args.warmup + i)
+        total_s += time_oracle(wl, inputs, r, cores)
+        total_pairs += pr
+        nrows += len(r)
+    value = total_pairs / total_s
+    sample = (f"each step: {nrows / args.steps:.1f} of {wl.T} query rows of {wl.name} "
+              f"(~{total_pairs // args.steps} valid pairs), fp64 scores + top-k")
+    return {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total_s / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(wl),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def workload_config(wl, extra=None):
+    c = {"workload": wl.name, "T": wl.T, "H": wl.H, "D": wl.D,
+         "index_topk": wl.index_topk,
+         "kv_dtype": "fp8_e4m3+e8m0/32" if wl.dtype == syn.DTYPE_FP8 else "bf16",
+         "mask": "positions" if wl.mode == syn.MODE_POSITIONS else "causal"}
+    if wl.mode == syn.MODE_POSITIONS:
+        c.update(S=wl.S, positions=f"U[{wl.pos_lo},{wl.pos_hi})",
+                 caches="shared" if wl.shared_cache else "one per token")
+    else:
+        c.update(seqlens=list(wl.seqlens))
+    if extra:
+        c.update(extra)
+    return c
+
+
+# ---------------------------------------------------------------- main
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=None)
+    ap.add_argument("--workload", default="decode_batch", choices=sorted(syn.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    wl = syn.WORKLOADS[args.workload]
+    d_steps, d_warm, _ = DEFAULTS[wl.name]
+    args.steps = d_steps if args.steps is None else args.steps
+    args.warmup = d_warm if args.warmup is None else args.warmup
+    if args.steps < 1 or args.warmup < 3:
+        ap.error("need --steps >= 1 and --warmup >= 3")
+    rank, world, local_rank = dist_env()
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, wl)), flush=True)
+        return 0
+
+    import torch
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    dist = init_dist(world, "nccl")
+    try:
+        r = run_ours(args, wl, dist, rank, world, device)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    pk = peaks()
+    value = r["pairs"] * world / (r["ms_step"] / 1e3)
+    tensor_bound = wl.mode == syn.MODE_CAUSAL or wl.shared_cache
+    if tensor_bound:
+        peak_t = pk["bf16"] * (2.0 if wl.dtype == syn.DTYPE_FP8 else 1.0)
+        achieved = r["flops"] / (r["ms_score"] / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
+                "frac": achieved / peak_t}
+    else:
+        achieved = r["sbytes"] / (r["ms_score"] / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
+                "frac": achieved / pk["hbm"]}
+    traffic = profiled_traffic(wl.name)
+    roof.update(traffic=traffic, kernel="score_bf16_kernel",
+                kernel_ms=r["ms_score"], peak_source=f"{pk['src']} (MEASURED_PEAKS.json)"
+                if pk["src"] == "measured" else "fallback")
+    t_roof = max(r["flops"] / (pk["bf16"] * (2.0 if wl.dtype == syn.DTYPE_FP8 else 1.0) * 1e12),
+                 (r["sbytes"] + r["tbytes"]) / (pk["hbm"] * 1e9))
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8" if wl.dtype == syn.DTYPE_FP8 else "bf16", "data": "synthetic",
+        "config": workload_config(wl, {
+            "l2": (f"{r['nsets']} rotating input copies" if r["nsets"] > 1
+                   else "inputs larger than L2"),
+            "steps_from": "CUDA graphs of forward calls",
+            "parallelism": f"{world} independent replicas" if world > 1 else "1 GPU"}),
+        "valid_pairs_per_step": r["pairs"],
+        "tflops": r["flops"] * world / (r["ms_step"] / 1e3) / 1e12,
+        "roofline": roof,
+        "path_roofline": {"roofline_ms": t_roof * 1e3, "step_ms": r["ms_step"],
+                          "frac": t_roof * 1e3 / r["ms_step"],
+                          "score_ms": r["ms_score"], "topk_ms": r["ms_topk"]},
+        "clocks": r["clocks"], "e2e": r["e2e"], "gpu_launches": 2 * args.steps,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(wl, syn.generate(wl))
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

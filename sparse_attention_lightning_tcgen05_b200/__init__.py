@@ -1,0 +1,144 @@
+"""Python binding of libdsa_indexer (the B200 lightning indexer).
+
+Argument marshalling only: every step of the indexer runs in the CUDA
+kernels of ``libdsa_indexer.so`` behind the C ABI of
+``include/dsa_indexer.h``. Names mirror the C entry points. PyTorch is used
+for device memory and streams; there is no CPU path. Importing this package
+raises if the library has not been built
+(``python -m sparse_attention_lightning_tcgen05_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdsa_indexer.so")
+
+DSA_OK = 0
+DSA_ERR_INVALID_ARG = 1
+DSA_ERR_UNSUPPORTED = 2
+DSA_ERR_WORKSPACE = 3
+DSA_ERR_CUDA = 4
+DSA_ERR_TIMEOUT = 5
+DSA_ERR_DEVICE = 6
+
+DSA_KV_BF16 = 0
+DSA_KV_FP8_E4M3_E8M0_B32 = 1
+DSA_MASK_POSITIONS = 0
+DSA_MASK_CAUSAL = 1
+DSA_MASK_BOUND = float.fromhex("-0x1.FEp127")
+
+# Every symbol include/dsa_indexer.h declares.
+EXPORTS = ("dsa_indexer_workspace_size", "dsa_indexer_score", "dsa_indexer_topk",
+           "dsa_indexer_forward", "dsa_indexer_get_error", "dsa_status_string")
+
+
+class dsa_indexer_desc_t(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32),
+                ("D", ctypes.c_int32), ("index_topk", ctypes.c_int32),
+                ("S", ctypes.c_int64), ("k_seq_stride", ctypes.c_int64),
+                ("num_seqs", ctypes.c_int32), ("cu_seqlens", ctypes.c_void_p),
+                ("dtype", ctypes.c_int), ("mask", ctypes.c_int)]
+
+
+class DsaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {dsa_status_string(status)}")
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with "
+        "'python -m sparse_attention_lightning_tcgen05_b200.build'")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_vp, _sz = ctypes.c_void_p, ctypes.c_size_t
+_P = ctypes.POINTER(dsa_indexer_desc_t)
+_lib.dsa_indexer_workspace_size.argtypes = [_P, ctypes.POINTER(_sz)]
+_lib.dsa_indexer_score.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.dsa_indexer_topk.argtypes = [_P, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.dsa_indexer_forward.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.dsa_indexer_get_error.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_int)]
+_lib.dsa_status_string.argtypes = [ctypes.c_int]
+_lib.dsa_status_string.restype = ctypes.c_char_p
+for _f in EXPORTS[:-1]:
+    getattr(_lib, _f).restype = ctypes.c_int
+
+
+def _ptr(x) -> int | None:
+    """A device pointer from a torch tensor, an int, or None."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def make_desc(T, H, index_topk, *, D=128, S=0, k_seq_stride=0, num_seqs=0,
+              cu_seqlens=None, dtype=DSA_KV_BF16, mask=DSA_MASK_POSITIONS):
+    return dsa_indexer_desc_t(T=T, H=H, D=D, index_topk=index_topk, S=S,
+                              k_seq_stride=k_seq_stride, num_seqs=num_seqs,
+                              cu_seqlens=_ptr(cu_seqlens), dtype=dtype,
+                              mask=mask)
+
+
+def dsa_status_string(status: int) -> str:
+    return _lib.dsa_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> int:
+    if status != DSA_OK:
+        raise DsaError(status, where)
+    return status
+
+
+def dsa_indexer_workspace_size(desc) -> int:
+    n = _sz(0)
+    _check(_lib.dsa_indexer_workspace_size(ctypes.byref(desc), ctypes.byref(n)),
+           "dsa_indexer_workspace_size")
+    return n.value
+
+
+def dsa_indexer_score(desc, q, q_scale, w, k, k_scale, positions, scores,
+                      workspace, workspace_bytes, stream=None) -> int:
+    return _check(_lib.dsa_indexer_score(
+        ctypes.byref(desc), _ptr(q), _ptr(q_scale), _ptr(w), _ptr(k),
+        _ptr(k_scale), _ptr(positions), _ptr(scores), _ptr(workspace),
+        workspace_bytes, stream), "dsa_indexer_score")
+
+
+def dsa_indexer_topk(desc, scores, positions, topk, workspace,
+                     workspace_bytes, stream=None) -> int:
+    return _check(_lib.dsa_indexer_topk(
+        ctypes.byref(desc), _ptr(scores), _ptr(positions), _ptr(topk),
+        _ptr(workspace), workspace_bytes, stream), "dsa_indexer_topk")
+
+
+def dsa_indexer_forward(desc, q, q_scale, w, k, k_scale, positions, scores,
+                        topk, workspace, workspace_bytes, stream=None) -> int:
+    return _check(_lib.dsa_indexer_forward(
+        ctypes.byref(desc), _ptr(q), _ptr(q_scale), _ptr(w), _ptr(k),
+        _ptr(k_scale), _ptr(positions), _ptr(scores), _ptr(topk),
+        _ptr(workspace), workspace_bytes, stream), "dsa_indexer_forward")
+
+
+def dsa_indexer_get_error(workspace, stream=None) -> int:
+    """Device-side status of the last call that used `workspace` (syncs)."""
+    st = ctypes.c_int(0)
+    _check(_lib.dsa_indexer_get_error(_ptr(workspace), stream, ctypes.byref(st)),
+           "dsa_indexer_get_error")
+    return st.value
+
+
+def raw_status(fn_name: str, *args) -> int:
+    """Call a C entry point and return its status code without raising
+    (for callers that inspect error codes)."""
+    return getattr(_lib, fn_name)(*args)
+
+
+def current_stream_handle():
+    """The cudaStream_t of torch's current CUDA stream."""
+    import torch
+    return torch.cuda.current_stream().cuda_stream

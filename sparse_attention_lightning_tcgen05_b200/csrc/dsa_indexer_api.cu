@@ -1,0 +1,353 @@
+// dsa_indexer_api.cu -- C ABI of libdsa_indexer: argument checks, TMA tensor
+// maps, kernel choice and launches. The operations, layouts and error rules
+// are stated in include/dsa_indexer.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "dsa_indexer.h"
+#include "score_kernel.cuh"
+#include "topk_kernel.cuh"
+
+namespace {
+
+using dsa::ScoreParams;
+using dsa::ScoreSmem;
+using dsa::TopkParams;
+
+constexpr size_t kWorkspaceHeader = 256;   // err, err_info, sched counter, ...
+constexpr uint64_t kWaitLimitNs = 4000000000ull;   // 4 s for any single wait
+constexpr int kMaxDevices = 64;
+constexpr uint32_t kMaxSmemPerBlock = 232448;      // 227 KB opt-in limit of sm_100
+
+// Words of the workspace header.
+// err/err_info: first device-side failure since the last get_error (sticky).
+// sched_counter/done_counter: score-kernel work scheduler; every launch
+// leaves them at zero when it exits.
+struct WsHeader {
+  unsigned int err;
+  unsigned int err_info;
+  unsigned int sched_counter;
+  unsigned int done_counter;
+  unsigned int pad[60];
+};
+static_assert(sizeof(WsHeader) == kWorkspaceHeader, "header size");
+
+// ---- per-device state -----------------------------------------------------------
+
+struct DeviceInfo {
+  bool probed = false;
+  bool ok = false;
+  int num_sms = 0;
+  uint32_t attr_done = 0;   // bit per kernel whose smem attribute is set
+};
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+dsa_status_t device_info(DeviceInfo **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return DSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo &d = g_dev[dev];
+  if (!d.probed) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    d.probed = true;
+    d.ok = (major == 10 && minor == 0);
+    d.num_sms = sms;
+  }
+  if (!d.ok) return DSA_ERR_DEVICE;
+  if (!g_encode) {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+      return DSA_ERR_CUDA;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  *out = &d;
+  return DSA_OK;
+}
+
+// Raise the dynamic shared-memory limit of kernel `bit` once per device.
+template <typename K>
+dsa_status_t ensure_smem_attr(DeviceInfo *d, uint32_t bit, K kernel, int bytes) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (d->attr_done >> bit & 1u) return DSA_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess)
+    return DSA_ERR_CUDA;
+  d->attr_done |= 1u << bit;
+  return DSA_OK;
+}
+
+// ---- argument checks -----------------------------------------------------------------
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+dsa_status_t check_desc(const dsa_indexer_desc_t *d) {
+  if (!d) return DSA_ERR_INVALID_ARG;
+  if (d->T < 1 || d->H < 1 || d->index_topk < 1) return DSA_ERR_INVALID_ARG;
+  if (d->dtype != DSA_KV_BF16 && d->dtype != DSA_KV_FP8_E4M3_E8M0_B32) return DSA_ERR_INVALID_ARG;
+  if (d->mask != DSA_MASK_POSITIONS && d->mask != DSA_MASK_CAUSAL) return DSA_ERR_INVALID_ARG;
+  if (d->D != 128) return DSA_ERR_UNSUPPORTED;
+  if (d->H > 256) return DSA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(d->T) * d->H > INT32_MAX - 256) return DSA_ERR_UNSUPPORTED;
+  if (d->mask == DSA_MASK_POSITIONS) {
+    if (d->S < 1) return DSA_ERR_INVALID_ARG;
+    if (d->S > INT32_MAX - 256) return DSA_ERR_UNSUPPORTED;
+    if (d->k_seq_stride != 0) {
+      if (d->k_seq_stride < d->S * d->D || d->k_seq_stride % d->D != 0) return DSA_ERR_INVALID_ARG;
+    }
+  } else {
+    if (d->num_seqs < 1 || !d->cu_seqlens) return DSA_ERR_INVALID_ARG;
+  }
+  if (d->dtype == DSA_KV_FP8_E4M3_E8M0_B32) return DSA_ERR_UNSUPPORTED;   // not built yet
+  return DSA_OK;
+}
+
+dsa_status_t check_workspace(const void *ws, size_t bytes) {
+  if (!ws || !aligned(ws, 256) || bytes < kWorkspaceHeader) return DSA_ERR_WORKSPACE;
+  return DSA_OK;
+}
+
+// ---- tensor maps -------------------------------------------------------------------------
+
+dsa_status_t make_map(CUtensorMap *m, CUtensorMapDataType dt, cuuint32_t rank, const void *base,
+                      const cuuint64_t *dims, const cuuint64_t *strides_bytes,
+                      const cuuint32_t *box) {
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, dt, rank, const_cast<void *>(base), dims, strides_bytes, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? DSA_OK : DSA_ERR_INVALID_ARG;
+}
+
+// One kernel choice: template instance, its sub-block geometry and chunking.
+struct ScoreLaunch {
+  void (*kernel)(const CUtensorMap, const CUtensorMap, const ScoreParams);
+  uint32_t attr_bit;
+  int stages, qbuf, nsub, threads;
+  int tq_sub, n_cols, chunk;
+  int max_cols;   // widest query block this instance ever runs (smem attribute)
+};
+
+int round16(int x) { return (x + 15) / 16 * 16; }
+
+ScoreLaunch choose_score(const dsa_indexer_desc_t *d) {
+  const bool per_token_cache = d->mask == DSA_MASK_POSITIONS && d->k_seq_stride != 0;
+  ScoreLaunch L{};
+  if (per_token_cache) {
+    if (d->H == 64) {
+      L = {dsa::score_bf16_kernel<64, 1, 4, 5, 2, 4>, 0, 5, 2, 1, 6 * 32, 1, 64, 4, 64};
+    } else {
+      L = {dsa::score_bf16_kernel<0, 1, 2, 4, 1, 4>, 1, 4, 1, 1, 6 * 32, 1, round16(d->H), 4, 256};
+    }
+  } else {
+    if (d->H == 64) {
+      L = {dsa::score_bf16_kernel<64, 2, 2, 2, 1, 8>, 2, 2, 1, 2, 10 * 32, 4, 256, 16, 256};
+    } else {
+      const int tq = 256 / d->H;
+      L = {dsa::score_bf16_kernel<0, 1, 2, 4, 1, 4>, 1, 4, 1, 1, 6 * 32, tq, round16(tq * d->H), 16, 256};
+    }
+  }
+  return L;
+}
+
+dsa_status_t launch_score(const dsa_indexer_desc_t *d, const void *q, const float *w,
+                          const void *k, const int32_t *positions, float *scores,
+                          WsHeader *ws, cudaStream_t stream) {
+  DeviceInfo *dev = nullptr;
+  dsa_status_t st = device_info(&dev);
+  if (st != DSA_OK) return st;
+  const ScoreLaunch L = choose_score(d);
+  const ScoreSmem plan(L.stages, L.qbuf, L.nsub, L.n_cols, false);
+  // the attribute is set once per kernel: use the widest query block it runs
+  const ScoreSmem widest(L.stages, L.qbuf, L.nsub, L.max_cols, false);
+  if (widest.total > kMaxSmemPerBlock || plan.total > widest.total) return DSA_ERR_UNSUPPORTED;
+  st = ensure_smem_attr(dev, L.attr_bit, L.kernel, static_cast<int>(widest.total));
+  if (st != DSA_OK) return st;
+
+  CUtensorMap tk, tq;
+  {
+    const bool causal = d->mask == DSA_MASK_CAUSAL;
+    const cuuint64_t rows = causal ? static_cast<cuuint64_t>(d->T) : static_cast<cuuint64_t>(d->S);
+    const cuuint64_t caches = (causal || d->k_seq_stride == 0) ? 1 : static_cast<cuuint64_t>(d->T);
+    const cuuint64_t zstride =
+        (causal || d->k_seq_stride == 0) ? rows * 256 : static_cast<cuuint64_t>(d->k_seq_stride) * 2;
+    const cuuint64_t dims[3] = {128, rows, caches};
+    const cuuint64_t strides[2] = {256, zstride};
+    const cuuint32_t box[3] = {64, dsa::kBlockM, 1};
+    st = make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, k, dims, strides, box);
+    if (st != DSA_OK) return st;
+  }
+  {
+    const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(d->T) * d->H};
+    const cuuint64_t strides[1] = {256};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(L.n_cols)};
+    st = make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, dims, strides, box);
+    if (st != DSA_OK) return st;
+  }
+
+  ScoreParams p{};
+  p.mode = d->mask == DSA_MASK_CAUSAL ? dsa::kModeCausal : dsa::kModePositions;
+  p.T = d->T;
+  p.H = d->H;
+  p.S = d->S;
+  p.shared_cache = d->k_seq_stride == 0;
+  p.num_seqs = d->num_seqs;
+  p.cu_seqlens = d->cu_seqlens;
+  p.positions = positions;
+  p.w = w;
+  p.scores = scores;
+  p.tq_sub = L.tq_sub;
+  p.n_cols = L.n_cols;
+  p.chunk_tiles = L.chunk;
+  p.sched_counter = &ws->sched_counter;
+  p.done_counter = &ws->done_counter;
+  p.err = &ws->err;
+  p.err_info = &ws->err_info;
+  p.wait_limit_ns = kWaitLimitNs;
+
+  int grid = dev->num_sms;
+  if (p.mode == dsa::kModePositions) {
+    const int64_t ntiles = (d->S + dsa::kBlockM - 1) / dsa::kBlockM;
+    const int64_t nch = (ntiles + L.chunk - 1) / L.chunk;
+    const int tq_total = L.tq_sub * L.nsub;
+    const int64_t nqb = p.shared_cache ? (d->T + tq_total - 1) / tq_total : d->T;
+    if (nqb * nch > UINT32_MAX / 2) return DSA_ERR_UNSUPPORTED;
+    if (nqb * nch < grid) grid = static_cast<int>(nqb * nch);
+  }
+  L.kernel<<<grid, L.threads, plan.total, stream>>>(tk, tq, p);
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+dsa_status_t launch_topk(const dsa_indexer_desc_t *d, const float *scores,
+                         const int32_t *positions, int32_t *topk, cudaStream_t stream) {
+  DeviceInfo *dev = nullptr;
+  dsa_status_t st = device_info(&dev);
+  if (st != DSA_OK) return st;
+  const int smem = static_cast<int>(sizeof(dsa::TopkSmem));
+  st = ensure_smem_attr(dev, 8, dsa::topk_kernel, smem);
+  if (st != DSA_OK) return st;
+  TopkParams p{};
+  p.mode = d->mask == DSA_MASK_CAUSAL ? dsa::kModeCausal : dsa::kModePositions;
+  p.T = d->T;
+  p.S = d->S;
+  p.num_seqs = d->num_seqs;
+  p.cu_seqlens = d->cu_seqlens;
+  p.positions = positions;
+  p.scores = scores;
+  p.topk = topk;
+  p.k = d->index_topk;
+  dsa::topk_kernel<<<d->T, dsa::kTopkThreads, smem, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+dsa_status_t check_inputs(const dsa_indexer_desc_t *d, const void *q, const uint8_t *q_scale,
+                          const float *w, const void *k, const uint8_t *k_scale,
+                          const int32_t *positions, const float *scores) {
+  if (!q || !w || !k || !scores) return DSA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(w, 16) || !aligned(scores, 4))
+    return DSA_ERR_INVALID_ARG;
+  if (d->mask == DSA_MASK_POSITIONS && !positions) return DSA_ERR_INVALID_ARG;
+  if (d->dtype == DSA_KV_FP8_E4M3_E8M0_B32 && (!q_scale || !k_scale)) return DSA_ERR_INVALID_ARG;
+  return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+dsa_status_t dsa_indexer_workspace_size(const dsa_indexer_desc_t *desc, size_t *bytes) {
+  if (!bytes) return DSA_ERR_INVALID_ARG;
+  const dsa_status_t st = check_desc(desc);
+  if (st != DSA_OK) return st;
+  *bytes = kWorkspaceHeader;
+  return DSA_OK;
+}
+
+dsa_status_t dsa_indexer_score(const dsa_indexer_desc_t *desc, const void *q,
+                               const uint8_t *q_scale, const float *w, const void *k,
+                               const uint8_t *k_scale, const int32_t *positions,
+                               float *scores, void *workspace, size_t workspace_bytes,
+                               dsa_stream_t stream) {
+  dsa_status_t st = check_desc(desc);
+  if (st == DSA_OK) st = check_inputs(desc, q, q_scale, w, k, k_scale, positions, scores);
+  if (st == DSA_OK) st = check_workspace(workspace, workspace_bytes);
+  if (st != DSA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return launch_score(desc, q, w, k, positions, scores, static_cast<WsHeader *>(workspace), s);
+}
+
+dsa_status_t dsa_indexer_topk(const dsa_indexer_desc_t *desc, const float *scores,
+                              const int32_t *positions, int32_t *topk, void *workspace,
+                              size_t workspace_bytes, dsa_stream_t stream) {
+  dsa_status_t st = check_desc(desc);
+  if (st != DSA_OK) return st;
+  if (!scores || !topk || !aligned(scores, 4) || !aligned(topk, 4)) return DSA_ERR_INVALID_ARG;
+  if (desc->mask == DSA_MASK_POSITIONS && !positions) return DSA_ERR_INVALID_ARG;
+  st = check_workspace(workspace, workspace_bytes);
+  if (st != DSA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return launch_topk(desc, scores, positions, topk, s);
+}
+
+dsa_status_t dsa_indexer_forward(const dsa_indexer_desc_t *desc, const void *q,
+                                 const uint8_t *q_scale, const float *w, const void *k,
+                                 const uint8_t *k_scale, const int32_t *positions,
+                                 float *scores, int32_t *topk, void *workspace,
+                                 size_t workspace_bytes, dsa_stream_t stream) {
+  dsa_status_t st = check_desc(desc);
+  if (st == DSA_OK) st = check_inputs(desc, q, q_scale, w, k, k_scale, positions, scores);
+  if (st == DSA_OK && (!topk || !aligned(topk, 4))) st = DSA_ERR_INVALID_ARG;
+  if (st == DSA_OK) st = check_workspace(workspace, workspace_bytes);
+  if (st != DSA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  st = launch_score(desc, q, w, k, positions, scores, static_cast<WsHeader *>(workspace), s);
+  if (st != DSA_OK) return st;
+  return launch_topk(desc, scores, positions, topk, s);
+}
+
+dsa_status_t dsa_indexer_get_error(const void *workspace, dsa_stream_t stream,
+                                   dsa_status_t *device_status) {
+  if (!workspace || !device_status || !aligned(workspace, 256)) return DSA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned int err = 0;
+  if (cudaMemcpyAsync(&err, workspace, sizeof err, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  // read and clear: the next report starts from a clean status
+  if (err != 0 && (cudaMemsetAsync(const_cast<void *>(workspace), 0, 2 * sizeof err, s) !=
+                       cudaSuccess ||
+                   cudaStreamSynchronize(s) != cudaSuccess))
+    return DSA_ERR_CUDA;
+  *device_status = err == 0 ? DSA_OK : static_cast<dsa_status_t>(err);
+  return DSA_OK;
+}
+
+const char *dsa_status_string(dsa_status_t status) {
+  switch (status) {
+    case DSA_OK: return "DSA_OK";
+    case DSA_ERR_INVALID_ARG: return "DSA_ERR_INVALID_ARG";
+    case DSA_ERR_UNSUPPORTED: return "DSA_ERR_UNSUPPORTED";
+    case DSA_ERR_WORKSPACE: return "DSA_ERR_WORKSPACE";
+    case DSA_ERR_CUDA: return "DSA_ERR_CUDA";
+    case DSA_ERR_TIMEOUT: return "DSA_ERR_TIMEOUT";
+    case DSA_ERR_DEVICE: return "DSA_ERR_DEVICE";
+  }
+  return "DSA_ERR_UNKNOWN";
+}
+
+}  // extern "C"

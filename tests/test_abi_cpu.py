@@ -1,0 +1,101 @@
+"""The C-ABI library loads, exports what include/dsa_indexer.h declares, and
+rejects bad arguments on the host before any device work (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_attention_lightning_tcgen05_b200 as dsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dsa_indexer.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(dsa_\w+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol():
+    names = declared_functions()
+    assert len(names) >= 6
+    lib = ctypes.CDLL(dsa.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(dsa.EXPORTS)
+
+
+def test_library_does_not_link_libcuda_or_torch():
+    # loads on a machine without a driver; cudart is linked statically
+    out = os.popen(f"ldd {dsa.LIB_PATH}").read()
+    assert "libcuda.so" not in out and "libtorch" not in out and "libc10" not in out
+
+
+def good_desc(**kw):
+    d = dict(T=4, H=64, index_topk=16, S=1024, k_seq_stride=1024 * 128)
+    d.update(kw)
+    return dsa.make_desc(**d)
+
+
+def test_workspace_size_on_host():
+    assert dsa.dsa_indexer_workspace_size(good_desc()) >= 256
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(T=0), dsa.DSA_ERR_INVALID_ARG),
+    (dict(H=0), dsa.DSA_ERR_INVALID_ARG),
+    (dict(index_topk=0), dsa.DSA_ERR_INVALID_ARG),
+    (dict(D=64), dsa.DSA_ERR_UNSUPPORTED),
+    (dict(H=300), dsa.DSA_ERR_UNSUPPORTED),
+    (dict(S=0), dsa.DSA_ERR_INVALID_ARG),
+    (dict(k_seq_stride=1000), dsa.DSA_ERR_INVALID_ARG),
+    (dict(k_seq_stride=1023 * 128), dsa.DSA_ERR_INVALID_ARG),
+    (dict(mask=dsa.DSA_MASK_CAUSAL, num_seqs=0), dsa.DSA_ERR_INVALID_ARG),
+    (dict(dtype=7), dsa.DSA_ERR_INVALID_ARG),
+])
+def test_bad_descriptors(kw, code):
+    with pytest.raises(dsa.DsaError) as e:
+        dsa.dsa_indexer_workspace_size(good_desc(**kw))
+    assert e.value.status == code
+
+
+def test_bad_pointers_rejected_before_device_work():
+    d = good_desc()
+    fake = 1 << 20                     # never dereferenced: checks fail first
+    with pytest.raises(dsa.DsaError) as e:
+        dsa.dsa_indexer_score(d, None, None, fake, fake, None, fake, fake, fake, 256)
+    assert e.value.status == dsa.DSA_ERR_INVALID_ARG
+    with pytest.raises(dsa.DsaError) as e:       # misaligned q
+        dsa.dsa_indexer_score(d, fake + 2, None, fake, fake, None, fake, fake, fake, 256)
+    assert e.value.status == dsa.DSA_ERR_INVALID_ARG
+    with pytest.raises(dsa.DsaError) as e:       # positions missing
+        dsa.dsa_indexer_forward(d, fake, None, fake, fake, None, None, fake, fake, fake, 256)
+    assert e.value.status == dsa.DSA_ERR_INVALID_ARG
+    with pytest.raises(dsa.DsaError) as e:       # workspace too small
+        dsa.dsa_indexer_forward(d, fake, None, fake, fake, None, fake, fake, fake, fake, 8)
+    assert e.value.status == dsa.DSA_ERR_WORKSPACE
+    with pytest.raises(dsa.DsaError) as e:       # workspace misaligned
+        dsa.dsa_indexer_topk(d, fake, fake, fake, fake + 16, 256)
+    assert e.value.status == dsa.DSA_ERR_WORKSPACE
+    with pytest.raises(dsa.DsaError) as e:       # no top-k output
+        dsa.dsa_indexer_topk(d, fake, fake, None, fake, 256)
+    assert e.value.status == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_status_strings():
+    for code in range(7):
+        assert dsa.dsa_status_string(code).startswith("DSA_")
+    assert dsa.dsa_status_string(99) == "DSA_ERR_UNKNOWN"
+
+
+def test_valid_call_without_a_gpu_fails_cleanly():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    fake = 1 << 20
+    with pytest.raises(dsa.DsaError) as e:
+        dsa.dsa_indexer_forward(good_desc(), fake, None, fake, fake, None, fake,
+                                fake, fake, fake, 256)
+    assert e.value.status == dsa.DSA_ERR_CUDA

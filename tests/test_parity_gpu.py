@@ -1,0 +1,132 @@
+"""CUDA path vs the fp64 oracle, through the C ABI (GPU only)."""
+import numpy as np
+import pytest
+import torch
+
+import dsa_synth as syn
+import oracle
+from parity_util import TOL_BF16, check_scores, check_topk, gpu_rows
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dsa():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import sparse_attention_lightning_tcgen05_b200 as m
+    from sparse_attention_lightning_tcgen05_b200.problem import DeviceProblem
+    return m, DeviceProblem
+
+
+def run_and_check(dsa, wl, inputs, rows=None, tol=TOL_BF16, exact=False):
+    m, DeviceProblem = dsa
+    dp = DeviceProblem.from_workload(wl, inputs)
+    dp.forward()
+    assert dp.device_status() == m.DSA_OK
+    torch.cuda.synchronize()
+    P = oracle.Problem(wl, inputs)
+    rows = list(range(wl.T)) if rows is None else [int(r) for r in rows]
+    orc = P.scores(rows)
+    gpu = gpu_rows(P, dp.scores, rows)
+    if exact:
+        for t, g, o in zip(rows, gpu, orc):
+            np.testing.assert_array_equal(g, o, err_msg=f"row {t}")
+    worst = check_scores(P, rows, gpu, orc, tol)
+    tk = dp.topk.cpu().numpy()[rows]
+    check_topk(P, rows, tk, gpu, orc, wl.index_topk, tol)
+    return worst
+
+
+def decode_wl(T=4, H=4, S=1024, k=64, shared=False, pos=(64, 1024), seed=0):
+    return syn.Workload("d", syn.MODE_POSITIONS, T=T, H=H, D=128, index_topk=k,
+                        S=S, shared_cache=shared, pos_lo=pos[0], pos_hi=pos[1],
+                        w_scale=1.0 / np.sqrt(H), seed=seed)
+
+
+def causal_wl(seqlens, H=64, k=64, seed=0):
+    return syn.Workload("c", syn.MODE_CAUSAL, T=int(sum(seqlens)), H=H, D=128,
+                        index_topk=k, seqlens=tuple(seqlens),
+                        w_scale=1.0 / np.sqrt(H), seed=seed)
+
+
+def test_tiny_decode_full(dsa):
+    wl = syn.WORKLOADS["tiny_decode"]
+    run_and_check(dsa, wl, syn.generate(wl))
+
+
+@pytest.mark.parametrize("H", [1, 4, 8, 16, 32, 64, 128])
+def test_decode_heads(dsa, H):
+    wl = decode_wl(T=3, H=H, S=700, k=100, pos=(0, 700), seed=H)
+    run_and_check(dsa, wl, syn.generate(wl))
+
+
+@pytest.mark.parametrize("H", [4, 64])
+def test_decode_integer_inputs_bit_exact(dsa, H):
+    wl = decode_wl(T=3, H=H, S=520, k=32, pos=(100, 520), seed=3)
+    run_and_check(dsa, wl, syn.generate(wl, value_kind="int"), exact=True)
+
+
+@pytest.mark.parametrize("H", [4, 64])
+def test_causal_integer_inputs_bit_exact(dsa, H):
+    wl = causal_wl((1, 130, 257), H=H, k=16, seed=4)
+    run_and_check(dsa, wl, syn.generate(wl, value_kind="int"), exact=True)
+
+
+def test_decode_position_edges(dsa):
+    """pos = 0, pos = S-1, pos >= S, negative pos, S not a multiple of 128."""
+    wl = decode_wl(T=6, H=64, S=333, k=40, seed=5)
+    inputs = syn.generate(wl)
+    inputs["positions"] = np.array([0, 332, 5000, -1, 127, 128], np.int32)
+    run_and_check(dsa, wl, inputs)
+
+
+def test_decode_shared_cache(dsa):
+    wl = decode_wl(T=11, H=64, S=900, k=50, shared=True, pos=(0, 900), seed=6)
+    run_and_check(dsa, wl, syn.generate(wl))
+
+
+def test_decode_shared_cache_generic_heads(dsa):
+    wl = decode_wl(T=70, H=4, S=300, k=20, shared=True, pos=(0, 300), seed=7)
+    run_and_check(dsa, wl, syn.generate(wl))
+
+
+@pytest.mark.parametrize("H", [1, 4, 16, 64])
+def test_causal_ragged_small(dsa, H):
+    wl = causal_wl((1, 7, 127, 128, 129, 300, 1000), H=H, k=64, seed=H)
+    run_and_check(dsa, wl, syn.generate(wl))
+
+
+def test_k_larger_than_rows(dsa):
+    wl = causal_wl((50, 3), H=64, k=2048, seed=8)
+    run_and_check(dsa, wl, syn.generate(wl))
+
+
+def test_topk_ties_integer_scores(dsa):
+    """Many exact ties (H=1 integer inputs): the tie rule picks the lower
+    slots, bit-exact."""
+    wl = causal_wl((600,), H=1, k=100, seed=9)
+    run_and_check(dsa, wl, syn.generate(wl, value_kind="int"), exact=True)
+
+
+def test_decode_batch_full_size(dsa):
+    wl = syn.WORKLOADS["decode_batch"]
+    run_and_check(dsa, wl, syn.generate(wl))
+
+
+def test_prefill_causal_full_size_sampled(dsa):
+    wl = syn.WORKLOADS["prefill_causal"]
+    rng = np.random.default_rng(11)
+    rows = [0, 1, 127, 128, 2046, 2047, 2048, 4095, 8191] + \
+        list(rng.integers(0, 8192, 12))
+    run_and_check(dsa, wl, syn.generate(wl), rows=rows)
+
+
+def test_ragged_prefill_full_size_sampled(dsa):
+    wl = syn.WORKLOADS["ragged_prefill"]
+    cu = wl.cu_seqlens()
+    rng = np.random.default_rng(12)
+    rows = []
+    for i in range(len(wl.seqlens)):
+        rows += [cu[i], cu[i] + 1, cu[i] + 2049, cu[i + 1] - 1]
+    rows += list(rng.integers(0, wl.T, 8))
+    run_and_check(dsa, wl, syn.generate(wl), rows=sorted(set(int(r) for r in rows)))

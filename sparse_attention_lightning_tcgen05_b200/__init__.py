@@ -5,7 +5,7 @@ kernels of ``libdsa_indexer.so`` behind the C ABI of
 ``include/dsa_indexer.h``. Names mirror the C entry points. PyTorch is used
 for device memory and streams; there is no CPU path. Importing this package
 raises if the library has not been built
-(``python -m sparse_attention_lightning_tcgen05_b200.build``).
+(``python sparse_attention_lightning_tcgen05_b200/build.py``).
 """
 from __future__ import annotations
 
@@ -48,12 +48,14 @@ class DsaError(RuntimeError):
         super().__init__(f"{where}: {dsa_status_string(status)}")
 
 
+_BUILD_HINT = "python sparse_attention_lightning_tcgen05_b200/build.py"
 if not os.path.exists(LIB_PATH):
-    raise ImportError(
-        f"{LIB_PATH} is missing: build it with "
-        "'python -m sparse_attention_lightning_tcgen05_b200.build'")
+    raise ImportError(f"{LIB_PATH} is missing: build it with '{_BUILD_HINT}'")
 
 _lib = ctypes.CDLL(LIB_PATH)
+for _f in EXPORTS:
+    if not hasattr(_lib, _f):
+        raise ImportError(f"{LIB_PATH} lacks {_f} (stale build): rebuild with '{_BUILD_HINT}'")
 _vp, _sz = ctypes.c_void_p, ctypes.c_size_t
 _P = ctypes.POINTER(dsa_indexer_desc_t)
 _lib.dsa_indexer_workspace_size.argtypes = [_P, ctypes.POINTER(_sz)]

@@ -1,6 +1,7 @@
 """Build libdsa_indexer.so in-tree with nvcc for sm_100a (no torch involved).
 
-Usage: python -m sparse_attention_lightning_tcgen05_b200.build [--force]
+Usage: python sparse_attention_lightning_tcgen05_b200/build.py [--force]
+(run it by path: importing the package loads the library it builds)
 """
 from __future__ import annotations
 

@@ -10,16 +10,16 @@
 #include <mutex>
 
 #include "dsa_indexer.h"
+#include "dsa_launch.h"
 #include "score_kernel.cuh"
 #include "topk_kernel.cuh"
 
-namespace {
+namespace dsa_host {
 
 using dsa::ScoreParams;
 using dsa::ScoreSmem;
 using dsa::TopkParams;
 
-constexpr size_t kWorkspaceHeader = 256;   // err, err_info, sched counter, ...
 constexpr uint64_t kWaitLimitNs = 4000000000ull;   // 4 s for any single wait
 constexpr int kMaxDevices = 64;
 constexpr uint32_t kMaxSmemPerBlock = 232448;      // 227 KB opt-in limit of sm_100
@@ -266,7 +266,9 @@ dsa_status_t check_inputs(const dsa_indexer_desc_t *d, const void *q, const uint
   return DSA_OK;
 }
 
-}  // namespace
+}  // namespace dsa_host
+
+using namespace dsa_host;
 
 extern "C" {
 

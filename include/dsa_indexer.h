@@ -156,6 +156,26 @@ dsa_status_t dsa_indexer_forward(const dsa_indexer_desc_t *desc,
                                  int32_t *topk, void *workspace,
                                  size_t workspace_bytes, dsa_stream_t stream);
 
+/* Forward pass (scores + top-k, as dsa_indexer_forward) that allocates
+ * nothing and takes no workspace. The pages have no counterpart: this entry
+ * point serves callers that cannot allocate device memory when they run the
+ * indexer (an engine plugin handed only its inputs and outputs, a runtime
+ * with a fixed memory pool, a path where an allocation could synchronise the
+ * device). The kernels' scratch words live in a fixed 4096-byte array inside
+ * the library, held by every GPU that loads it until the process exits; a
+ * problem whose workspace size exceeds it returns DSA_ERR_WORKSPACE. The
+ * first call on a device looks up that array's address (do it before any
+ * stream capture). Every call clears the scratch on `stream`; all calls share
+ * it, so calls that overlap on the GPU race and must be serialised by the
+ * caller. Device-side timeouts are not reported by this entry point. */
+dsa_status_t dsa_indexer_forward_noalloc(const dsa_indexer_desc_t *desc,
+                                         const void *q, const uint8_t *q_scale,
+                                         const float *w, const void *k,
+                                         const uint8_t *k_scale,
+                                         const int32_t *positions,
+                                         float *scores, int32_t *topk,
+                                         dsa_stream_t stream);
+
 /* Synchronises `stream`, then reports in *device_status the first
  * device-side failure (DSA_ERR_TIMEOUT) recorded in `workspace` since the
  * previous dsa_indexer_get_error on it, or DSA_OK, and clears it. Returns

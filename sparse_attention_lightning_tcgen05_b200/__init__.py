@@ -31,7 +31,8 @@ DSA_MASK_BOUND = float.fromhex("-0x1.FEp127")
 
 # Every symbol include/dsa_indexer.h declares.
 EXPORTS = ("dsa_indexer_workspace_size", "dsa_indexer_score", "dsa_indexer_topk",
-           "dsa_indexer_forward", "dsa_indexer_get_error", "dsa_status_string")
+           "dsa_indexer_forward", "dsa_indexer_forward_noalloc",
+           "dsa_indexer_get_error", "dsa_status_string")
 
 
 class dsa_indexer_desc_t(ctypes.Structure):
@@ -62,6 +63,7 @@ _lib.dsa_indexer_workspace_size.argtypes = [_P, ctypes.POINTER(_sz)]
 _lib.dsa_indexer_score.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.dsa_indexer_topk.argtypes = [_P, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.dsa_indexer_forward.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+_lib.dsa_indexer_forward_noalloc.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.dsa_indexer_get_error.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_int)]
 _lib.dsa_status_string.argtypes = [ctypes.c_int]
 _lib.dsa_status_string.restype = ctypes.c_char_p
@@ -124,6 +126,17 @@ def dsa_indexer_forward(desc, q, q_scale, w, k, k_scale, positions, scores,
         ctypes.byref(desc), _ptr(q), _ptr(q_scale), _ptr(w), _ptr(k),
         _ptr(k_scale), _ptr(positions), _ptr(scores), _ptr(topk),
         _ptr(workspace), workspace_bytes, stream), "dsa_indexer_forward")
+
+
+def dsa_indexer_forward_noalloc(desc, q, q_scale, w, k, k_scale, positions,
+                                scores, topk, stream=None) -> int:
+    """dsa_indexer_forward without a workspace: for callers that cannot
+    allocate device memory; the library's fixed scratch is used instead
+    (calls must not overlap on the GPU)."""
+    return _check(_lib.dsa_indexer_forward_noalloc(
+        ctypes.byref(desc), _ptr(q), _ptr(q_scale), _ptr(w), _ptr(k),
+        _ptr(k_scale), _ptr(positions), _ptr(scores), _ptr(topk), stream),
+        "dsa_indexer_forward_noalloc")
 
 
 def dsa_indexer_get_error(workspace, stream=None) -> int:

@@ -99,3 +99,15 @@ def test_valid_call_without_a_gpu_fails_cleanly():
         dsa.dsa_indexer_forward(good_desc(), fake, None, fake, fake, None, fake,
                                 fake, fake, fake, 256)
     assert e.value.status == dsa.DSA_ERR_CUDA
+
+
+def test_noalloc_rejects_bad_arguments_on_the_host():
+    fake = 1 << 20
+    with pytest.raises(dsa.DsaError) as e:       # no top-k output
+        dsa.dsa_indexer_forward_noalloc(good_desc(), fake, None, fake, fake, None,
+                                        fake, fake, None)
+    assert e.value.status == dsa.DSA_ERR_INVALID_ARG
+    with pytest.raises(dsa.DsaError) as e:
+        dsa.dsa_indexer_forward_noalloc(good_desc(D=64), fake, None, fake, fake, None,
+                                        fake, fake, fake)
+    assert e.value.status == dsa.DSA_ERR_UNSUPPORTED

@@ -21,6 +21,7 @@ queries == keys, head_dim == 128, block-32 e8m0 scales).
 from __future__ import annotations
 
 import dataclasses
+import os
 from typing import Optional
 
 import numpy as np
@@ -131,7 +132,8 @@ def f32_to_mx_e4m3(x: np.ndarray):
     floored at 448 * 2^-127 so that e >= -127); byte = e + 127. Each element is
     then x * 2^-e rounded to the nearest e4m3 value, ties to even (|x * 2^-e|
     <= 448, so nothing saturates). Returns (data uint8 [..., D], scale uint8
-    [..., D/32]).
+    [..., D/32]). Row chunks are encoded on a thread pool; every step is exact
+    power-of-two arithmetic, so the result does not depend on the chunking.
     """
     x = np.ascontiguousarray(x, dtype=np.float32)
     D = x.shape[-1]
@@ -140,17 +142,28 @@ def f32_to_mx_e4m3(x: np.ndarray):
     blocks = x.reshape(-1, D // MX_BLOCK, MX_BLOCK)
     data = np.empty(blocks.shape, dtype=np.uint8)
     scale = np.empty(blocks.shape[:2], dtype=np.uint8)
-    step = max(1, (1 << 22) // D)
-    for i in range(0, blocks.shape[0], step):
-        b = blocks[i:i + step].astype(np.float64)
-        amax = np.maximum(np.abs(b).max(axis=-1), E4M3_MAX * 2.0 ** -127)
+    step = max(1, (1 << 20) // D)
+
+    def work(i):
+        b = blocks[i:i + step]
+        amax = np.maximum(np.abs(b).max(axis=-1).astype(np.float64),
+                          E4M3_MAX * 2.0 ** -127)
         m, E = np.frexp(amax)                    # amax = m * 2^E, m in [0.5, 1)
         # 448 = 0.875 * 2^9: 448 * 2^e >= m * 2^E  <=>  e >= E - 9 + log2(m/0.875)
         e = E.astype(np.int64) - 9 + (m > 0.875)
         assert e.min() >= -127 and e.max() <= 127
         scale[i:i + step] = (e + 127).astype(np.uint8)
-        y = np.ldexp(b, -e[..., None])           # exact power-of-two scaling
+        y = np.ldexp(b.astype(np.float64), -e[..., None])   # exact scaling
         data[i:i + step] = _e4m3_rne_bytes(y)
+
+    starts = range(0, blocks.shape[0], step)
+    if blocks.shape[0] > 4 * step:
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(max_workers=os.cpu_count() or 1) as ex:
+            list(ex.map(work, starts))
+    else:
+        for i in starts:
+            work(i)
     return data.reshape(lead + (D,)), scale.reshape(lead + (D // MX_BLOCK,))
 
 

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -26,14 +27,10 @@ constexpr uint32_t kMaxSmemPerBlock = 232448;      // 227 KB opt-in limit of sm_
 
 // Words of the workspace header.
 // err/err_info: first device-side failure since the last get_error (sticky).
-// sched_counter/done_counter: score-kernel work scheduler; every launch
-// leaves them at zero when it exits.
 struct WsHeader {
   unsigned int err;
   unsigned int err_info;
-  unsigned int sched_counter;
-  unsigned int done_counter;
-  unsigned int pad[60];
+  unsigned int reserved[62];
 };
 static_assert(sizeof(WsHeader) == kWorkspaceHeader, "header size");
 
@@ -112,7 +109,11 @@ dsa_status_t check_desc(const dsa_indexer_desc_t *d) {
   } else {
     if (d->num_seqs < 1 || !d->cu_seqlens) return DSA_ERR_INVALID_ARG;
   }
-  if (d->dtype == DSA_KV_FP8_E4M3_E8M0_B32) return DSA_ERR_UNSUPPORTED;   // not built yet
+  if (d->dtype == DSA_KV_FP8_E4M3_E8M0_B32) {
+    if (d->H > 128) return DSA_ERR_UNSUPPORTED;
+    // scale rows of consecutive caches must start on 16-byte boundaries
+    if (d->mask == DSA_MASK_POSITIONS && d->k_seq_stride % 512 != 0) return DSA_ERR_INVALID_ARG;
+  }
   return DSA_OK;
 }
 
@@ -125,83 +126,127 @@ dsa_status_t check_workspace(const void *ws, size_t bytes) {
 
 dsa_status_t make_map(CUtensorMap *m, CUtensorMapDataType dt, cuuint32_t rank, const void *base,
                       const cuuint64_t *dims, const cuuint64_t *strides_bytes,
-                      const cuuint32_t *box) {
+                      const cuuint32_t *box,
+                      CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(m, dt, rank, const_cast<void *>(base), dims, strides_bytes, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? DSA_OK : DSA_ERR_INVALID_ARG;
 }
 
-// One kernel choice: template instance, its sub-block geometry and chunking.
+// One kernel choice: template instance, its sub-block geometry.
+using ScoreKernelFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                               const CUtensorMap, const ScoreParams);
 struct ScoreLaunch {
-  void (*kernel)(const CUtensorMap, const CUtensorMap, const ScoreParams);
+  ScoreKernelFn kernel;
   uint32_t attr_bit;
   int stages, qbuf, nsub, threads;
-  int tq_sub, n_cols, chunk;
+  int tq_sub, n_cols;
   int max_cols;   // widest query block this instance ever runs (smem attribute)
+  bool fp8;
 };
 
 int round16(int x) { return (x + 15) / 16 * 16; }
 
-ScoreLaunch choose_score(const dsa_indexer_desc_t *d) {
-  const bool per_token_cache = d->mask == DSA_MASK_POSITIONS && d->k_seq_stride != 0;
-  ScoreLaunch L{};
-  if (per_token_cache) {
-    if (d->H == 64) {
-      L = {dsa::score_bf16_kernel<64, 1, 4, 5, 2, 4>, 0, 5, 2, 1, 6 * 32, 1, 64, 4, 64};
-    } else {
-      L = {dsa::score_bf16_kernel<0, 1, 2, 4, 1, 4>, 1, 4, 1, 1, 6 * 32, 1, round16(d->H), 4, 256};
-    }
-  } else {
-    if (d->H == 64) {
-      L = {dsa::score_bf16_kernel<64, 2, 2, 2, 1, 8>, 2, 2, 1, 2, 10 * 32, 4, 256, 16, 256};
-    } else {
-      const int tq = 256 / d->H;
-      L = {dsa::score_bf16_kernel<0, 1, 2, 4, 1, 4>, 1, 4, 1, 1, 6 * 32, tq, round16(tq * d->H), 16, 256};
-    }
-  }
-  return L;
+// Largest power of two <= x (x >= 1).
+int pow2_floor(int x) {
+  int p = 1;
+  while (p * 2 <= x) p *= 2;
+  return p;
 }
 
-dsa_status_t launch_score(const dsa_indexer_desc_t *d, const void *q, const float *w,
-                          const void *k, const int32_t *positions, float *scores,
-                          WsHeader *ws, cudaStream_t stream) {
+ScoreLaunch choose_score(const dsa_indexer_desc_t *d) {
+  const bool per_token_cache = d->mask == DSA_MASK_POSITIONS && d->k_seq_stride != 0;
+  const int H = d->H;
+  if (d->dtype == DSA_KV_BF16) {
+    if (per_token_cache) {
+      if (H == 64)
+        return {dsa::score_kernel<64, 1, 4, 5, 2, 4, false>, 0, 5, 2, 1, 6 * 32, 1, 64, 64, false};
+      return {dsa::score_kernel<0, 1, 2, 4, 1, 4, false>, 1, 4, 1, 1, 6 * 32, 1, round16(H), 256,
+              false};
+    }
+    if (H == 64)
+      return {dsa::score_kernel<64, 2, 2, 2, 1, 8, false>, 2, 2, 1, 2, 10 * 32, 4, 256, 256, false};
+    const int tq = pow2_floor(std::min(128, 256 / H));
+    return {dsa::score_kernel<0, 1, 2, 4, 1, 4, false>, 1, 4, 1, 1, 6 * 32, tq, round16(tq * H), 256,
+            false};
+  }
+  if (per_token_cache) {
+    if (H == 64)
+      return {dsa::score_kernel<64, 1, 4, 8, 2, 4, true>, 3, 8, 2, 1, 6 * 32, 1, 64, 64, true};
+    return {dsa::score_kernel<0, 1, 2, 4, 1, 4, true>, 4, 4, 1, 1, 6 * 32, 1, round16(H), 128, true};
+  }
+  if (H == 64)
+    return {dsa::score_kernel<64, 2, 2, 4, 1, 8, true>, 5, 4, 1, 2, 10 * 32, 2, 128, 128, true};
+  const int tq = pow2_floor(std::min(128, 128 / H));
+  return {dsa::score_kernel<0, 1, 2, 4, 1, 4, true>, 4, 4, 1, 1, 6 * 32, tq, round16(tq * H), 128,
+          true};
+}
+
+dsa_status_t launch_score(const dsa_indexer_desc_t *d, const void *q, const uint8_t *q_scale,
+                          const float *w, const void *k, const uint8_t *k_scale,
+                          const int32_t *positions, float *scores, WsHeader *ws,
+                          cudaStream_t stream) {
   DeviceInfo *dev = nullptr;
   dsa_status_t st = device_info(&dev);
   if (st != DSA_OK) return st;
   const ScoreLaunch L = choose_score(d);
-  const ScoreSmem plan(L.stages, L.qbuf, L.nsub, L.n_cols, false);
+  const ScoreSmem plan(L.stages, L.qbuf, L.nsub, L.n_cols, L.fp8);
   // the attribute is set once per kernel: use the widest query block it runs
-  const ScoreSmem widest(L.stages, L.qbuf, L.nsub, L.max_cols, false);
+  const ScoreSmem widest(L.stages, L.qbuf, L.nsub, L.max_cols, L.fp8);
   if (widest.total > kMaxSmemPerBlock || plan.total > widest.total) return DSA_ERR_UNSUPPORTED;
   st = ensure_smem_attr(dev, L.attr_bit, L.kernel, static_cast<int>(widest.total));
   if (st != DSA_OK) return st;
 
-  CUtensorMap tk, tq;
+  const bool causal = d->mask == DSA_MASK_CAUSAL;
+  const bool shared = causal || d->k_seq_stride == 0;
+  const cuuint64_t rows = causal ? static_cast<cuuint64_t>(d->T) : static_cast<cuuint64_t>(d->S);
+  const cuuint64_t caches = shared ? 1 : static_cast<cuuint64_t>(d->T);
+  const cuuint64_t elt = L.fp8 ? 1 : 2;
+  const cuuint64_t stride_elems = shared ? rows * 128 : static_cast<cuuint64_t>(d->k_seq_stride);
+  const cuuint64_t qrows = static_cast<cuuint64_t>(d->T) * d->H;
+  CUtensorMap tk, tq, tksf, tqsf;
+  std::memset(&tksf, 0, sizeof tksf);
+  std::memset(&tqsf, 0, sizeof tqsf);
   {
-    const bool causal = d->mask == DSA_MASK_CAUSAL;
-    const cuuint64_t rows = causal ? static_cast<cuuint64_t>(d->T) : static_cast<cuuint64_t>(d->S);
-    const cuuint64_t caches = (causal || d->k_seq_stride == 0) ? 1 : static_cast<cuuint64_t>(d->T);
-    const cuuint64_t zstride =
-        (causal || d->k_seq_stride == 0) ? rows * 256 : static_cast<cuuint64_t>(d->k_seq_stride) * 2;
     const cuuint64_t dims[3] = {128, rows, caches};
-    const cuuint64_t strides[2] = {256, zstride};
-    const cuuint32_t box[3] = {64, dsa::kBlockM, 1};
-    st = make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, k, dims, strides, box);
+    const cuuint64_t strides[2] = {128 * elt, stride_elems * elt};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elt), dsa::kBlockM, 1};
+    st = make_map(&tk, L.fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                  k, dims, strides, box);
     if (st != DSA_OK) return st;
   }
   {
-    const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(d->T) * d->H};
-    const cuuint64_t strides[1] = {256};
-    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(L.n_cols)};
-    st = make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, dims, strides, box);
+    const cuuint64_t dims[2] = {128, qrows};
+    const cuuint64_t strides[1] = {128 * elt};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elt),
+                               static_cast<cuuint32_t>(L.n_cols)};
+    st = make_map(&tq, L.fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  q, dims, strides, box);
+    if (st != DSA_OK) return st;
+  }
+  if (L.fp8) {
+    // scale bytes of one slot (4 blocks of 32 along D) read as one 32-bit word
+    // (one cache: the second dimension is never stepped; its stride only
+    // has to be a legal multiple of 16 bytes)
+    const cuuint64_t dims[2] = {rows, caches};
+    const cuuint64_t strides[1] = {shared ? (rows * 4 + 15) / 16 * 16 : stride_elems / 32};
+    const cuuint32_t box[2] = {dsa::kBlockM + dsa::kSfPad, 1};
+    st = make_map(&tksf, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, k_scale, dims, strides, box,
+                  CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != DSA_OK) return st;
+    const cuuint64_t qdims[2] = {qrows, 1};
+    const cuuint64_t qstrides[1] = {(qrows * 4 + 15) / 16 * 16};   // never stepped
+    const cuuint32_t qbox[2] = {static_cast<cuuint32_t>(L.n_cols + dsa::kSfPad), 1};
+    st = make_map(&tqsf, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, q_scale, qdims, qstrides, qbox,
+                  CU_TENSOR_MAP_SWIZZLE_NONE);
     if (st != DSA_OK) return st;
   }
 
   ScoreParams p{};
-  p.mode = d->mask == DSA_MASK_CAUSAL ? dsa::kModeCausal : dsa::kModePositions;
+  p.mode = causal ? dsa::kModeCausal : dsa::kModePositions;
   p.T = d->T;
   p.H = d->H;
   p.S = d->S;
@@ -213,23 +258,18 @@ dsa_status_t launch_score(const dsa_indexer_desc_t *d, const void *q, const floa
   p.scores = scores;
   p.tq_sub = L.tq_sub;
   p.n_cols = L.n_cols;
-  p.chunk_tiles = L.chunk;
-  p.sched_counter = &ws->sched_counter;
-  p.done_counter = &ws->done_counter;
   p.err = &ws->err;
   p.err_info = &ws->err_info;
   p.wait_limit_ns = kWaitLimitNs;
 
   int grid = dev->num_sms;
-  if (p.mode == dsa::kModePositions) {
+  if (!causal) {
     const int64_t ntiles = (d->S + dsa::kBlockM - 1) / dsa::kBlockM;
-    const int64_t nch = (ntiles + L.chunk - 1) / L.chunk;
-    const int tq_total = L.tq_sub * L.nsub;
-    const int64_t nqb = p.shared_cache ? (d->T + tq_total - 1) / tq_total : d->T;
-    if (nqb * nch > UINT32_MAX / 2) return DSA_ERR_UNSUPPORTED;
-    if (nqb * nch < grid) grid = static_cast<int>(nqb * nch);
+    const int tqt = L.tq_sub * L.nsub;
+    const int64_t nqb = p.shared_cache ? (d->T + tqt - 1) / tqt : d->T;
+    if (nqb * ntiles < grid) grid = static_cast<int>(nqb * ntiles);
   }
-  L.kernel<<<grid, L.threads, plan.total, stream>>>(tk, tq, p);
+  L.kernel<<<grid, L.threads, plan.total, stream>>>(tk, tq, tksf, tqsf, p);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
@@ -290,7 +330,8 @@ dsa_status_t dsa_indexer_score(const dsa_indexer_desc_t *desc, const void *q,
   if (st == DSA_OK) st = check_workspace(workspace, workspace_bytes);
   if (st != DSA_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  return launch_score(desc, q, w, k, positions, scores, static_cast<WsHeader *>(workspace), s);
+  return launch_score(desc, q, q_scale, w, k, k_scale, positions, scores,
+                      static_cast<WsHeader *>(workspace), s);
 }
 
 dsa_status_t dsa_indexer_topk(const dsa_indexer_desc_t *desc, const float *scores,
@@ -317,7 +358,8 @@ dsa_status_t dsa_indexer_forward(const dsa_indexer_desc_t *desc, const void *q,
   if (st == DSA_OK) st = check_workspace(workspace, workspace_bytes);
   if (st != DSA_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  st = launch_score(desc, q, w, k, positions, scores, static_cast<WsHeader *>(workspace), s);
+  st = launch_score(desc, q, q_scale, w, k, k_scale, positions, scores,
+                    static_cast<WsHeader *>(workspace), s);
   if (st != DSA_OK) return st;
   return launch_topk(desc, scores, positions, topk, s);
 }

@@ -7,7 +7,7 @@
 // memory pool and forbids allocations after start-up, or a path that must not
 // allocate because allocation can synchronise the device. This entry point
 // runs the same score and top-k kernels as dsa_indexer_forward, but the
-// scratch words those kernels need (error word, work-scheduler counters) live
+// scratch words those kernels need (the device-side error word and site) live
 // in a fixed array compiled into the library instead of a caller workspace.
 //
 // The array is a file-scope __device__ variable of kNoAllocScratchBytes: every
@@ -75,7 +75,7 @@ extern "C" dsa_status_t dsa_indexer_forward_noalloc(
   if (st != DSA_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(scratch, 0, need, s) != cudaSuccess) return DSA_ERR_CUDA;
-  st = dsa_host::launch_score(desc, q, w, k, positions, scores,
+  st = dsa_host::launch_score(desc, q, q_scale, w, k, k_scale, positions, scores,
                               static_cast<dsa_host::WsHeader *>(scratch), s);
   if (st != DSA_OK) return st;
   return dsa_host::launch_topk(desc, scores, positions, topk, s);

@@ -20,9 +20,10 @@ dsa_status_t check_desc(const dsa_indexer_desc_t *d);
 dsa_status_t check_inputs(const dsa_indexer_desc_t *d, const void *q, const uint8_t *q_scale,
                           const float *w, const void *k, const uint8_t *k_scale,
                           const int32_t *positions, const float *scores);
-dsa_status_t launch_score(const dsa_indexer_desc_t *d, const void *q, const float *w,
-                          const void *k, const int32_t *positions, float *scores,
-                          WsHeader *ws, cudaStream_t stream);
+dsa_status_t launch_score(const dsa_indexer_desc_t *d, const void *q, const uint8_t *q_scale,
+                          const float *w, const void *k, const uint8_t *k_scale,
+                          const int32_t *positions, float *scores, WsHeader *ws,
+                          cudaStream_t stream);
 dsa_status_t launch_topk(const dsa_indexer_desc_t *d, const float *scores,
                          const int32_t *positions, int32_t *topk, cudaStream_t stream);
 

@@ -10,18 +10,27 @@
 // the epilogue is thread-local: no shuffles, and a warp's 32 lanes write 32
 // consecutive scores of a row.
 //
-//   warp 0      : work scheduler + TMA producer (one elected thread)
-//   warp 1      : TMEM allocator + MMA issuer (one elected thread)
+//   warp 0      : TMA producer (one thread)
+//   warp 1      : TMEM allocator + MMA issuer (one thread issues; for fp8 the
+//                 whole warp first lays the scale factors out for tcgen05.cp)
 //   warps 2..   : epilogue (TMEM -> ReLU, w-weighted head sum, mask, store)
 //
-// Work unit = (query block of up to tq_sub*NSUB tokens sharing one key
-// cache, range of `chunk_tiles` key tiles). Units are handed out through a
-// global atomic counter and a small shared-memory ring so that the three
-// roles walk the same sequence. Per active key tile the MMA issues one
-// accumulator per sub-block (NSUB); accumulators rotate through NACC TMEM
-// buffers so the epilogue of one overlaps the MMA of the next. Key tiles past
-// every token's last valid slot are never loaded: the epilogue writes the
-// mask bound there directly.
+// Schedule: a query block is up to tq_sub*NSUB consecutive tokens that read
+// one key cache. An "active item" is (query block, key tile) with the tile
+// holding at least one valid slot of the block; a "fill item" is a tile of the
+// block's score rows where every slot is masked. Both lists are split into
+// equal contiguous ranges, one per CTA (no atomics, balanced to one tile).
+// Per active item the MMA issues one accumulator per sub-block; accumulators
+// rotate through NACC TMEM buffers so the epilogue of one overlaps the MMA of
+// the next. Fill items are never loaded: the epilogue writes the mask bound,
+// before it turns to its active items.
+//
+// fp8 (MX) variant: e4m3 q and k with one e8m0 scale per 32 elements along D
+// (Sparse Attention Indexer MX BF16Score Kernel API Reference: block-32 e8m0
+// scales). The scales are applied inside the MMA
+// (tcgen05.mma kind::mxf8f6f4.block_scale): TMA brings the scale words next to
+// the data, the MMA warp reorders them into the 128-row scale-factor atom and
+// copies them into TMEM with tcgen05.cp; no dequantised copy is ever written.
 #pragma once
 
 #include <cstdint>
@@ -32,7 +41,6 @@ namespace dsa {
 
 constexpr int kBlockM = 128;          // key slots per tile (MMA M)
 constexpr int kHeadDim = 128;         // D
-constexpr int kSchedSlots = 4;        // unit ring depth
 constexpr float kMaskBound = -0x1.FEp127f;   // lowest finite bf16
 
 enum : int { kModePositions = 0, kModeCausal = 1 };
@@ -47,115 +55,339 @@ struct ScoreParams {
   const int *positions;      // POSITIONS
   const float *w;            // [T, H]
   float *scores;
-  int tq_sub;                // tokens per MMA sub-block
+  int tq_sub;                // tokens per MMA sub-block (tq_sub*NSUB divides 128)
   int n_cols;                // MMA N per sub-block: round_up(tq_sub*H, 16)
-  int chunk_tiles;           // key tiles per work unit
-  unsigned int *sched_counter;   // next unit to hand out (0 at launch)
-  unsigned int *done_counter;    // CTAs finished (0 at launch)
   unsigned int *err;
   unsigned int *err_info;
   uint64_t wait_limit_ns;
 };
 
+__host__ __device__ constexpr int sf_atoms(int n_cols) { return (n_cols + 127) / 128; }
+
+// fp8 scale windows: TMA loads scale words from a start rounded down to a
+// multiple of 4 words (a tiled copy of 32-bit elements must start 16-byte
+// aligned along its innermost dimension), so every window holds 4 extra words.
+// Every TMA destination in shared memory starts on a 128-byte boundary, so
+// the windows' sizes are rounded up to 128 bytes.
+constexpr int kSfPad = 4;
+__host__ __device__ constexpr uint32_t round128(uint32_t x) { return (x + 127u) & ~127u; }
+// bytes one scale-window copy delivers (the mbarrier's expected transaction
+// count) and the shared-memory room it takes
+constexpr uint32_t kSfBoxBytesK = (kBlockM + kSfPad) * 4;
+constexpr uint32_t kSfRawBytesK = round128(kSfBoxBytesK);
+__host__ __device__ constexpr uint32_t sf_box_bytes_q(int n_cols) {
+  return static_cast<uint32_t>((n_cols + kSfPad) * 4);
+}
+__host__ __device__ constexpr uint32_t sf_raw_bytes_q(int n_cols) {
+  return round128(sf_box_bytes_q(n_cols));
+}
+
 // Shared-memory plan, identical on host and device.
 struct ScoreSmem {
-  uint32_t k_stage_bytes, q_sub_bytes;
-  uint32_t off_k, off_q, off_bar, off_misc, total;
-  __host__ __device__ ScoreSmem(int stages, int qbuf, int nsub, int n_cols,
-                                bool fp8) {
+  uint32_t k_stage_bytes, k_sf_bytes, q_sub_bytes, q_sf_bytes;
+  uint32_t off_k, off_ksf, off_q, off_qsf, off_bar, off_misc, total;
+  __host__ __device__ ScoreSmem(int stages, int qbuf, int nsub, int n_cols, bool fp8) {
     // bf16: two 128-byte-wide halves along D; fp8: one 128-byte row.
     k_stage_bytes = fp8 ? kBlockM * 128 : kBlockM * 256;
     q_sub_bytes = fp8 ? n_cols * 128 : n_cols * 256;
+    // fp8 scale words (4 bytes a row) as loaded -- a window of rows + 4 words
+    // that starts at a multiple of 4 words, the TMA alignment rule for 32-bit
+    // elements -- followed by the reordered atoms (512 B each).
+    k_sf_bytes = fp8 ? kSfRawBytesK + 512 : 0;
+    q_sf_bytes = fp8 ? static_cast<uint32_t>(sf_raw_bytes_q(n_cols) + sf_atoms(n_cols) * 512) : 0;
     off_k = 0;
     off_q = off_k + stages * k_stage_bytes;
-    off_bar = off_q + qbuf * nsub * q_sub_bytes;
+    off_ksf = off_q + qbuf * nsub * q_sub_bytes;
+    off_qsf = off_ksf + stages * k_sf_bytes;
+    off_bar = off_qsf + qbuf * nsub * q_sf_bytes;
+    off_bar = (off_bar + 15) & ~15u;
     off_misc = off_bar + 64 * 8;            // up to 64 mbarriers
-    total = off_misc + 128 + 1024;          // misc words + alignment slack
+    total = off_misc + 256 + 1024;          // misc words + alignment slack
   }
 };
 
-struct Unit {
+// TMEM columns: accumulators, then (fp8) per-stage A scales, then per
+// query-buffer sub-block B scales.
+__host__ __device__ constexpr int tmem_cols_needed(int nacc, int n_cols, int stages,
+                                                  int qbuf, int nsub, bool fp8) {
+  return nacc * n_cols + (fp8 ? stages * 4 + qbuf * nsub * 4 * sf_atoms(n_cols) : 0);
+}
+
+// ---- the static schedule --------------------------------------------------------
+
+// One query block and the key tiles of its score rows.
+struct QBlk {
+  int seq, b;          // CAUSAL: sequence and block in it; POSITIONS: seq 0, block b
   int t0, ntok;        // tokens [t0, t0 + ntok)
-  int z;               // key-cache index (3rd TMA coordinate)
-  int y0;              // first key row of the sequence (2nd TMA coordinate)
+  int z, y0;           // key cache (3rd TMA coordinate), first key row (2nd)
   int64_t row_len;     // slots per score row
   int64_t out0;        // float offset of token t0's score row
+  int64_t seqoff;      // CAUSAL: float offset of the sequence's score block
   int lv0;             // CAUSAL: last valid slot of token t0
-  int j0, j1;          // key tiles [j0, j1) of this unit
-  int j_act;           // tiles [j0, j_act) need the MMA; [j_act, j1) are masked
+  int act, ntr;        // tiles holding a valid slot; tiles in the row
 };
 
 __device__ __forceinline__ int last_valid_pos(const ScoreParams &p, int t) {
-  int pos = __ldg(p.positions + t);
-  int64_t lv = pos < 0 ? -1 : (pos >= p.S ? p.S - 1 : pos);
+  const int pos = __ldg(p.positions + t);
+  const int64_t lv = pos < 0 ? -1 : (pos >= p.S ? p.S - 1 : pos);
   return static_cast<int>(lv);
 }
 
-// Last valid slot of token t0 + i of unit U.
-__device__ __forceinline__ int unit_last_valid(const ScoreParams &p,
-                                               const Unit &U, int i) {
-  return p.mode == kModeCausal ? U.lv0 + i : last_valid_pos(p, U.t0 + i);
+// Last valid slot of token t0 + i of block q.
+__device__ __forceinline__ int qb_last_valid(const ScoreParams &p, const QBlk &q, int i) {
+  return p.mode == kModeCausal ? q.lv0 + i : last_valid_pos(p, q.t0 + i);
 }
 
-// Decode work unit u. Returns false once u is past the last unit. Every
-// role calls this with the same u and gets the same answer.
-__device__ bool decode_unit(const ScoreParams &p, int tq_total, uint32_t u,
-                            Unit &U) {
-  const int ch = p.chunk_tiles;
+__device__ __forceinline__ int pos_num_blocks(const ScoreParams &p, int tqt) {
+  return p.shared_cache ? (p.T + tqt - 1) / tqt : p.T;
+}
+
+__device__ void make_qb_positions(const ScoreParams &p, int tqt, int b, QBlk &q) {
+  q.seq = 0;
+  q.b = b;
+  q.t0 = b * tqt;
+  q.ntok = min(tqt, p.T - q.t0);
+  q.z = p.shared_cache ? 0 : q.t0;
+  q.y0 = 0;
+  q.row_len = p.S;
+  q.out0 = static_cast<int64_t>(q.t0) * p.S;
+  q.seqoff = 0;
+  q.lv0 = 0;
+  int mx = -1;
+  for (int i = 0; i < q.ntok; ++i) mx = max(mx, last_valid_pos(p, q.t0 + i));
+  q.ntr = static_cast<int>((p.S + kBlockM - 1) / kBlockM);
+  q.act = mx < 0 ? 0 : mx / kBlockM + 1;
+}
+
+__device__ void make_qb_causal(const ScoreParams &p, int tqt, int seq, int b,
+                               int64_t seqoff, QBlk &q) {
+  const int a = __ldg(p.cu_seqlens + seq);
+  const int L = __ldg(p.cu_seqlens + seq + 1) - a;
+  const int tl0 = b * tqt;
+  q.seq = seq;
+  q.b = b;
+  q.t0 = a + tl0;
+  q.ntok = min(tqt, L - tl0);
+  q.z = 0;
+  q.y0 = a;
+  q.row_len = L;
+  q.seqoff = seqoff;
+  q.out0 = seqoff + static_cast<int64_t>(tl0) * L;
+  q.lv0 = tl0;
+  q.ntr = (L + kBlockM - 1) / kBlockM;
+  q.act = (tl0 + q.ntok - 1) / kBlockM + 1;
+}
+
+// CAUSAL, tqt dividing 128: block b of a sequence has floor(b/r) + 1 active
+// tiles (r = 128/tqt), so the active tiles of blocks [0, B) number
+// B + r*m*(m-1)/2 + m*(B - m*r) with m = B / r.
+__device__ __forceinline__ int64_t causal_active_before(int64_t B, int r) {
+  const int64_t m = B / r, rem = B - m * r;
+  return B + r * m * (m - 1) / 2 + m * rem;
+}
+
+// Move q to the next query block (skipping empty sequences). False at the end.
+__device__ bool next_qb(const ScoreParams &p, int tqt, QBlk &q) {
   if (p.mode == kModePositions) {
-    const int64_t ntiles = (p.S + kBlockM - 1) / kBlockM;
-    const int64_t nch = (ntiles + ch - 1) / ch;
-    const int64_t nqb = p.shared_cache ? (p.T + tq_total - 1) / tq_total : p.T;
-    if (static_cast<int64_t>(u) >= nqb * nch) return false;
-    const int64_t c = u / nqb, qb = u % nqb;     // chunk-major: early slots first
-    U.t0 = static_cast<int>(qb * tq_total);
-    U.ntok = min(tq_total, p.T - U.t0);
-    U.z = p.shared_cache ? 0 : U.t0;
-    U.y0 = 0;
-    U.row_len = p.S;
-    U.out0 = static_cast<int64_t>(U.t0) * p.S;
-    U.lv0 = 0;
-    U.j0 = static_cast<int>(c * ch);
-    U.j1 = static_cast<int>(U.j0 + ch < ntiles ? U.j0 + ch : ntiles);
-    int mx = -1;
-    for (int i = 0; i < U.ntok; ++i) mx = max(mx, last_valid_pos(p, U.t0 + i));
-    U.j_act = mx < 0 ? U.j0 : min(U.j1, mx / kBlockM + 1);
-    U.j_act = max(U.j_act, U.j0);
+    if (q.b + 1 >= pos_num_blocks(p, tqt)) return false;
+    make_qb_positions(p, tqt, q.b + 1, q);
     return true;
   }
-  // CAUSAL: sequences in order; inside one, the longest query blocks first.
-  int64_t uu = u, seqoff = 0;
-  for (int i = 0; i < p.num_seqs; ++i) {
-    const int a = __ldg(p.cu_seqlens + i), b = __ldg(p.cu_seqlens + i + 1);
-    const int L = b - a;
-    if (L <= 0) continue;
-    const int64_t nqb = (L + tq_total - 1) / tq_total;
-    const int64_t ntiles = (L + kBlockM - 1) / kBlockM;
-    const int64_t nch = (ntiles + ch - 1) / ch;
-    if (uu < nqb * nch) {
-      const int64_t blk = nqb - 1 - uu / nch, c = uu % nch;
-      const int tl0 = static_cast<int>(blk * tq_total);
-      U.t0 = a + tl0;
-      U.ntok = min(tq_total, L - tl0);
-      U.z = 0;
-      U.y0 = a;
-      U.row_len = L;
-      U.out0 = seqoff + static_cast<int64_t>(tl0) * L;
-      U.lv0 = tl0;
-      U.j0 = static_cast<int>(c * ch);
-      U.j1 = static_cast<int>(U.j0 + ch < ntiles ? U.j0 + ch : ntiles);
-      const int mx = tl0 + U.ntok - 1;
-      U.j_act = max(U.j0, min(U.j1, mx / kBlockM + 1));
+  const int L = static_cast<int>(q.row_len);
+  if ((q.b + 1) * tqt < L) {
+    make_qb_causal(p, tqt, q.seq, q.b + 1, q.seqoff, q);
+    return true;
+  }
+  int64_t off = q.seqoff + static_cast<int64_t>(L) * L;
+  for (int s = q.seq + 1; s < p.num_seqs; ++s) {
+    const int Ls = __ldg(p.cu_seqlens + s + 1) - __ldg(p.cu_seqlens + s);
+    if (Ls > 0) {
+      make_qb_causal(p, tqt, s, 0, off, q);
       return true;
     }
-    uu -= nqb * nch;
-    seqoff += static_cast<int64_t>(L) * L;
   }
   return false;
 }
 
-// Epilogue for one token with H == 64 (the tuned head count): the two
-// 32-column TMEM loads hold heads 0..31 and 32..63 of this slot.
+// Where a CTA starts: its shares of the active and fill lists, and the
+// (block, tile) of the first item of each.
+struct CtaRange {
+  int64_t a_count, f_count;
+  int a_seq, a_b, a_j;
+  int f_seq, f_b, f_j;
+  int64_t a_seqoff, f_seqoff;
+};
+
+// Inclusive warp scan of 64-bit counts.
+__device__ __forceinline__ int64_t warp_incl_scan64(int64_t v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int64_t n = __shfl_up_sync(0xffffffffu, v, off);
+    if (lane >= off) v += n;
+  }
+  return v;
+}
+
+// POSITIONS: the block holding item `idx` of the active (fill == false) or
+// fill list, by a warp-wide scan over blocks. Executed by a full warp.
+__device__ void locate_positions(const ScoreParams &p, int tqt, int64_t idx, bool fill,
+                                 int &b_out, int &j_out) {
+  const int lane = threadIdx.x & 31;
+  const int nqb = pos_num_blocks(p, tqt);
+  int64_t base = 0;
+  b_out = nqb;
+  j_out = 0;
+  for (int c0 = 0; c0 < nqb; c0 += 32) {
+    const int b = c0 + lane;
+    int64_t cnt = 0;
+    int act = 0;
+    if (b < nqb) {
+      QBlk q;
+      make_qb_positions(p, tqt, b, q);
+      act = q.act;
+      cnt = fill ? q.ntr - q.act : q.act;
+    }
+    const int64_t incl = warp_incl_scan64(cnt);
+    const int64_t total = __shfl_sync(0xffffffffu, incl, 31);
+    const unsigned hit = __ballot_sync(0xffffffffu, base + incl > idx);
+    if (hit) {
+      const int f = __ffs(hit) - 1;
+      const int64_t excl = __shfl_sync(0xffffffffu, incl - cnt, f);
+      const int act_f = __shfl_sync(0xffffffffu, act, f);
+      b_out = c0 + f;
+      j_out = static_cast<int>(idx - base - excl) + (fill ? act_f : 0);
+      return;
+    }
+    base += total;
+  }
+}
+
+// POSITIONS: total active and fill items (full warp).
+__device__ void count_positions(const ScoreParams &p, int tqt, int64_t &A, int64_t &F) {
+  const int lane = threadIdx.x & 31;
+  const int nqb = pos_num_blocks(p, tqt);
+  int64_t a = 0, f = 0;
+  for (int b = lane; b < nqb; b += 32) {
+    QBlk q;
+    make_qb_positions(p, tqt, b, q);
+    a += q.act;
+    f += q.ntr - q.act;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    a += __shfl_xor_sync(0xffffffffu, a, off);
+    f += __shfl_xor_sync(0xffffffffu, f, off);
+  }
+  A = a;
+  F = f;
+}
+
+// CAUSAL: active or fill items before block B of a sequence.
+__device__ __forceinline__ int64_t causal_before(int64_t B, int r, int ntr, bool fill) {
+  const int64_t a = causal_active_before(B, r);
+  return fill ? B * ntr - a : a;
+}
+
+// CAUSAL: locate item idx of the active or fill list (one thread).
+__device__ void locate_causal(const ScoreParams &p, int tqt, int64_t idx, bool fill,
+                              int &seq_out, int &b_out, int &j_out, int64_t &seqoff_out) {
+  const int r = kBlockM / tqt;
+  int64_t off = 0;
+  for (int s = 0; s < p.num_seqs; ++s) {
+    const int L = __ldg(p.cu_seqlens + s + 1) - __ldg(p.cu_seqlens + s);
+    if (L <= 0) continue;
+    const int nqb = (L + tqt - 1) / tqt, ntr = (L + kBlockM - 1) / kBlockM;
+    const int64_t tot = causal_before(nqb, r, ntr, fill);
+    if (idx < tot) {
+      int lo = 0, hi = nqb - 1;                 // last block whose prefix <= idx
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) / 2;
+        if (causal_before(mid, r, ntr, fill) <= idx) lo = mid; else hi = mid - 1;
+      }
+      seq_out = s;
+      b_out = lo;
+      j_out = static_cast<int>(idx - causal_before(lo, r, ntr, fill)) + (fill ? lo / r + 1 : 0);
+      seqoff_out = off;
+      return;
+    }
+    idx -= tot;
+    off += static_cast<int64_t>(L) * L;
+  }
+  seq_out = p.num_seqs;
+  b_out = 0;
+  j_out = 0;
+  seqoff_out = off;
+}
+
+__device__ void count_causal(const ScoreParams &p, int tqt, int64_t &A, int64_t &F) {
+  const int r = kBlockM / tqt;
+  A = 0;
+  F = 0;
+  for (int s = 0; s < p.num_seqs; ++s) {
+    const int L = __ldg(p.cu_seqlens + s + 1) - __ldg(p.cu_seqlens + s);
+    if (L <= 0) continue;
+    const int nqb = (L + tqt - 1) / tqt, ntr = (L + kBlockM - 1) / kBlockM;
+    A += causal_before(nqb, r, ntr, false);
+    F += causal_before(nqb, r, ntr, true);
+  }
+}
+
+// This CTA's share of both lists (executed by a full warp; every lane gets
+// the same result).
+__device__ void cta_range(const ScoreParams &p, int tqt, CtaRange &R) {
+  const int64_t G = gridDim.x, c = blockIdx.x;
+  int64_t A = 0, F = 0;
+  if (p.mode == kModePositions) count_positions(p, tqt, A, F);
+  else count_causal(p, tqt, A, F);
+  const int64_t a0 = A * c / G, a1 = A * (c + 1) / G;
+  const int64_t f0 = F * c / G, f1 = F * (c + 1) / G;
+  R.a_count = a1 - a0;
+  R.f_count = f1 - f0;
+  R.a_seq = R.f_seq = 0;
+  R.a_b = R.f_b = 0;
+  R.a_j = R.f_j = 0;
+  R.a_seqoff = R.f_seqoff = 0;
+  if (p.mode == kModePositions) {
+    if (R.a_count > 0) locate_positions(p, tqt, a0, false, R.a_b, R.a_j);
+    if (R.f_count > 0) locate_positions(p, tqt, f0, true, R.f_b, R.f_j);
+  } else {
+    if (R.a_count > 0) locate_causal(p, tqt, a0, false, R.a_seq, R.a_b, R.a_j, R.a_seqoff);
+    if (R.f_count > 0) locate_causal(p, tqt, f0, true, R.f_seq, R.f_b, R.f_j, R.f_seqoff);
+  }
+}
+
+__device__ __forceinline__ void make_qb(const ScoreParams &p, int tqt, int seq, int b,
+                                        int64_t seqoff, QBlk &q) {
+  if (p.mode == kModePositions) make_qb_positions(p, tqt, b, q);
+  else make_qb_causal(p, tqt, seq, b, seqoff, q);
+}
+
+// Advance an active cursor by one item: the next tile, or the first tile of
+// the next block that has one. False past the end of the list.
+__device__ __forceinline__ bool next_active(const ScoreParams &p, int tqt, QBlk &q, int &j) {
+  if (++j < q.act) return true;
+  do {
+    if (!next_qb(p, tqt, q)) return false;
+  } while (q.act == 0);
+  j = 0;
+  return true;
+}
+
+// Advance a fill cursor by one item.
+__device__ __forceinline__ bool next_fill(const ScoreParams &p, int tqt, QBlk &q, int &j) {
+  if (++j < q.ntr) return true;
+  do {
+    if (!next_qb(p, tqt, q)) return false;
+  } while (q.act == q.ntr);
+  j = q.act;
+  return true;
+}
+
+// ---- epilogue helpers ---------------------------------------------------------------
+
+// One token with H == 64 (the tuned head count): the two 32-column TMEM
+// loads hold heads 0..31 and 32..63 of this slot.
 __device__ __forceinline__ float head_sum_h64(uint32_t taddr, const float *wrow) {
   float v[32];
   float acc = 0.f;
@@ -183,24 +415,44 @@ struct Ring {
   }
 };
 
+// fp8: reorder 128 rows of 4 scale bytes (row-major, as loaded) into the
+// scale-factor atom tcgen05.cp copies: row m = m0 + 32*m1 at byte
+// 16*m0 + 4*m1 (+ K block). Rows >= nrows read as 0. Full warp.
+__device__ __forceinline__ void sf_reorder_atom(const uint32_t *rows, int nrows,
+                                                uint32_t *atom) {
+  const int l = threadIdx.x & 31;
+  uint4 v;
+  v.x = l < nrows ? rows[l] : 0u;
+  v.y = l + 32 < nrows ? rows[l + 32] : 0u;
+  v.z = l + 64 < nrows ? rows[l + 64] : 0u;
+  v.w = l + 96 < nrows ? rows[l + 96] : 0u;
+  reinterpret_cast<uint4 *>(atom)[l] = v;
+}
+
 // kH: 64 selects the tuned epilogue; 0 = any H (generic epilogue).
 // kNSUB: MMA sub-blocks per key tile (each its own accumulator, same A).
 // kNACC: TMEM accumulator buffers. kSTAGES: key-tile smem stages.
 // kQBUF: query-block smem buffers. kEPI: epilogue warps (4 or 8).
-template <int kH, int kNSUB, int kNACC, int kSTAGES, int kQBUF, int kEPI>
+// kFP8: e4m3 + e8m0/32 inputs through the block-scaled MMA.
+template <int kH, int kNSUB, int kNACC, int kSTAGES, int kQBUF, int kEPI, bool kFP8>
 __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
-    score_bf16_kernel(const __grid_constant__ CUtensorMap tmap_k,
-                      const __grid_constant__ CUtensorMap tmap_q,
-                      const ScoreParams p) {
+    score_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                 const __grid_constant__ CUtensorMap tmap_q,
+                 const __grid_constant__ CUtensorMap tmap_ksf,
+                 const __grid_constant__ CUtensorMap tmap_qsf,
+                 const ScoreParams p) {
   static_assert(kEPI == 4 || kEPI == 8, "epilogue warps");
   static_assert(kH == 64 || kEPI == 4, "generic epilogue uses 4 warps");
+  static_assert(2 * (kSTAGES + kQBUF + kNACC) <= 64, "barrier budget");
   constexpr int kGroups = kEPI / 4;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const ScoreSmem L(kSTAGES, kQBUF, kNSUB, p.n_cols, false);
+  const ScoreSmem L(kSTAGES, kQBUF, kNSUB, p.n_cols, kFP8);
   uint8_t *sk = smem + L.off_k;
   uint8_t *sq = smem + L.off_q;
+  uint8_t *sksf = smem + L.off_ksf;
+  uint8_t *sqsf = smem + L.off_qsf;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.off_bar);
   uint64_t *full_k = bars;                       // [kSTAGES]
   uint64_t *empty_k = full_k + kSTAGES;          // [kSTAGES]
@@ -208,35 +460,39 @@ __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
   uint64_t *q_empty = q_full + kQBUF;            // [kQBUF]
   uint64_t *acc_full = q_empty + kQBUF;          // [kNACC]
   uint64_t *acc_empty = acc_full + kNACC;        // [kNACC]
-  uint64_t *sched_full = acc_empty + kNACC;      // [kSchedSlots]
-  uint64_t *sched_empty = sched_full + kSchedSlots;
   uint32_t *misc = reinterpret_cast<uint32_t *>(smem + L.off_misc);
   uint32_t *tmem_base_slot = misc;               // written by tcgen05.alloc
   volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 1);
-  uint32_t *sched_unit = misc + 4;               // [kSchedSlots]
+  CtaRange *range_slot = reinterpret_cast<CtaRange *>(misc + 16);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const int tq_total = p.tq_sub * kNSUB;
+  const int tqt = p.tq_sub * kNSUB;              // tokens per query block
   const int n_cols = p.n_cols;
-  const uint32_t tmem_cols_needed = kNACC * n_cols;
+  const int atoms = sf_atoms(n_cols);
   uint32_t tmem_cols = 32;
-  while (tmem_cols < tmem_cols_needed) tmem_cols <<= 1;
+  while (tmem_cols < static_cast<uint32_t>(
+                         tmem_cols_needed(kNACC, n_cols, kSTAGES, kQBUF, kNSUB, kFP8)))
+    tmem_cols <<= 1;
 
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kSTAGES; ++i) { mbar_init(full_k + i, 1); mbar_init(empty_k + i, 1); }
-    for (int i = 0; i < kQBUF; ++i) { mbar_init(q_full + i, 1); mbar_init(q_empty + i, 1); }
-    for (int i = 0; i < kNACC; ++i) { mbar_init(acc_full + i, 1); mbar_init(acc_empty + i, kEPI); }
-    for (int i = 0; i < kSchedSlots; ++i) {
-      mbar_init(sched_full + i, 1);
-      mbar_init(sched_empty + i, 1 + kEPI);
+  if (warp == 0) {
+    CtaRange R;
+    cta_range(p, tqt, R);
+    if (lane == 0) {
+      *range_slot = R;
+      for (int i = 0; i < kSTAGES; ++i) { mbar_init(full_k + i, 1); mbar_init(empty_k + i, 1); }
+      for (int i = 0; i < kQBUF; ++i) { mbar_init(q_full + i, 1); mbar_init(q_empty + i, 1); }
+      for (int i = 0; i < kNACC; ++i) { mbar_init(acc_full + i, 1); mbar_init(acc_empty + i, kEPI); }
+      *abort_flag = 0;
+      fence_mbar_init();
+      tma_prefetch_desc(&tmap_k);
+      tma_prefetch_desc(&tmap_q);
+      if constexpr (kFP8) {
+        tma_prefetch_desc(&tmap_ksf);
+        tma_prefetch_desc(&tmap_qsf);
+      }
     }
-    *abort_flag = 0;
-    fence_mbar_init();
-    tma_prefetch_desc(&tmap_k);
-    tma_prefetch_desc(&tmap_q);
-  }
-  if (warp == 1) {
+  } else if (warp == 1) {
     tmem_alloc(tmem_base_slot, tmem_cols);
     tmem_relinquish();
   }
@@ -244,48 +500,62 @@ __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_base_slot;
+  const CtaRange R = *range_slot;
   const WaitCtl ctl{abort_flag, p.err, p.err_info, p.wait_limit_ns};
+  const uint32_t sfa_col0 = kNACC * n_cols;                    // fp8 only
+  const uint32_t sfb_col0 = sfa_col0 + kSTAGES * 4;            // fp8 only
 
   if (warp == 0) {
-    // ---------------- scheduler + TMA producer ----------------
-    if (lane == 0) {
-      Ring st, qb, sc;
-      uint32_t k_issued = 0, q_issued = 0;   // bitmasks: stage / buffer used
-      uint32_t k_last_phase = 0, q_last_phase = 0;
-      for (;;) {
-        const uint32_t u = atomicAdd(p.sched_counter, 1u);
-        if (!mbar_wait(sched_empty + sc.idx, sc.phase ^ 1u, ctl, 1)) break;
-        sched_unit[sc.idx] = u;
-        mbar_arrive(sched_full + sc.idx);
-        sc.next(kSchedSlots);
-        Unit U;
-        if (!decode_unit(p, tq_total, u, U)) break;
-        if (U.j_act == U.j0) continue;
-        const int nsub = (U.ntok + p.tq_sub - 1) / p.tq_sub;
-        if (!mbar_wait(q_empty + qb.idx, qb.phase ^ 1u, ctl, 2)) break;
-        mbar_arrive_expect_tx(q_full + qb.idx, nsub * L.q_sub_bytes);
-        for (int s = 0; s < nsub; ++s) {
-          uint8_t *dst = sq + (qb.idx * kNSUB + s) * L.q_sub_bytes;
-          const int row = (U.t0 + s * p.tq_sub) * p.H;
-          tma_load_2d(dst, &tmap_q, q_full + qb.idx, 0, row);
-          tma_load_2d(dst + n_cols * 128, &tmap_q, q_full + qb.idx, 64, row);
+    // ---------------- TMA producer ----------------
+    if (lane == 0 && R.a_count > 0) {
+      Ring st, qb;
+      uint32_t k_issued = 0, q_issued = 0, k_last_phase = 0, q_last_phase = 0;
+      QBlk q;
+      int j = R.a_j;
+      make_qb(p, tqt, R.a_seq, R.a_b, R.a_seqoff, q);
+      bool need_q = true;
+      for (int64_t n = 0; n < R.a_count; ++n) {
+        if (need_q) {
+          const int nsub = (q.ntok + p.tq_sub - 1) / p.tq_sub;
+          if (!mbar_wait(q_empty + qb.idx, qb.phase ^ 1u, ctl, 2)) break;
+          mbar_arrive_expect_tx(q_full + qb.idx,
+                                nsub * (L.q_sub_bytes + (kFP8 ? sf_box_bytes_q(n_cols) : 0)));
+          for (int s = 0; s < nsub; ++s) {
+            uint8_t *dst = sq + (qb.idx * kNSUB + s) * L.q_sub_bytes;
+            const int row = (q.t0 + s * p.tq_sub) * p.H;
+            if constexpr (kFP8) {
+              tma_load_2d(dst, &tmap_q, q_full + qb.idx, 0, row);
+              tma_load_2d(sqsf + (qb.idx * kNSUB + s) * L.q_sf_bytes, &tmap_qsf,
+                          q_full + qb.idx, row & ~(kSfPad - 1), 0);
+            } else {
+              tma_load_2d(dst, &tmap_q, q_full + qb.idx, 0, row);
+              tma_load_2d(dst + n_cols * 128, &tmap_q, q_full + qb.idx, 64, row);
+            }
+          }
+          q_issued |= 1u << qb.idx;
+          q_last_phase = (q_last_phase & ~(1u << qb.idx)) | (qb.phase << qb.idx);
+          need_q = false;
         }
-        q_issued |= 1u << qb.idx;
-        q_last_phase = (q_last_phase & ~(1u << qb.idx)) | (qb.phase << qb.idx);
-        qb.next(kQBUF);
-        bool ok = true;
-        for (int j = U.j0; j < U.j_act; ++j) {
-          if (!mbar_wait(empty_k + st.idx, st.phase ^ 1u, ctl, 3)) { ok = false; break; }
-          mbar_arrive_expect_tx(full_k + st.idx, L.k_stage_bytes);
-          uint8_t *dst = sk + st.idx * L.k_stage_bytes;
-          tma_load_3d(dst, &tmap_k, full_k + st.idx, 0, U.y0 + j * kBlockM, U.z);
-          tma_load_3d(dst + kBlockM * 128, &tmap_k, full_k + st.idx, 64,
-                      U.y0 + j * kBlockM, U.z);
-          k_issued |= 1u << st.idx;
-          k_last_phase = (k_last_phase & ~(1u << st.idx)) | (st.phase << st.idx);
-          st.next(kSTAGES);
+        if (!mbar_wait(empty_k + st.idx, st.phase ^ 1u, ctl, 3)) break;
+        mbar_arrive_expect_tx(full_k + st.idx, L.k_stage_bytes + (kFP8 ? kSfBoxBytesK : 0));
+        uint8_t *dst = sk + st.idx * L.k_stage_bytes;
+        const int y = q.y0 + j * kBlockM;
+        if constexpr (kFP8) {
+          tma_load_3d(dst, &tmap_k, full_k + st.idx, 0, y, q.z);
+          tma_load_2d(sksf + st.idx * L.k_sf_bytes, &tmap_ksf, full_k + st.idx,
+                      y & ~(kSfPad - 1), q.z);
+        } else {
+          tma_load_3d(dst, &tmap_k, full_k + st.idx, 0, y, q.z);
+          tma_load_3d(dst + kBlockM * 128, &tmap_k, full_k + st.idx, 64, y, q.z);
         }
-        if (!ok) break;
+        k_issued |= 1u << st.idx;
+        k_last_phase = (k_last_phase & ~(1u << st.idx)) | (st.phase << st.idx);
+        st.next(kSTAGES);
+        if (n + 1 < R.a_count) {
+          const int pb = q.b, ps = q.seq;
+          next_active(p, tqt, q, j);
+          if (q.b != pb || q.seq != ps) { need_q = true; qb.next(kQBUF); }
+        }
       }
       // Let every copy this thread started land before the CTA can exit.
       for (int i = 0; i < kSTAGES; ++i)
@@ -294,56 +564,115 @@ __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
         if (q_issued >> i & 1u) mbar_drain(q_full + i, q_last_phase >> i & 1u, p.wait_limit_ns);
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(kBlockM, n_cols);
-      Ring st, qb, ac, sc;
+    // ---------------- MMA issuer (whole warp walks the list) ----------------
+    if (R.a_count > 0) {
+      Ring st, qb, ac;
       uint64_t *last_commit = nullptr;
       uint32_t last_commit_phase = 0;
-      for (;;) {
-        if (!mbar_wait(sched_full + sc.idx, sc.phase, ctl, 11)) break;
-        const uint32_t u = sched_unit[sc.idx];
-        mbar_arrive(sched_empty + sc.idx);
-        sc.next(kSchedSlots);
-        Unit U;
-        if (!decode_unit(p, tq_total, u, U)) break;
-        if (U.j_act == U.j0) continue;
-        const int nsub = (U.ntok + p.tq_sub - 1) / p.tq_sub;
-        if (!mbar_wait(q_full + qb.idx, qb.phase, ctl, 12)) break;
+      QBlk q;
+      int j = R.a_j;
+      make_qb(p, tqt, R.a_seq, R.a_b, R.a_seqoff, q);
+      bool new_q = true;
+      for (int64_t n = 0; n < R.a_count; ++n) {
+        const int nsub = (q.ntok + p.tq_sub - 1) / p.tq_sub;
+        if (new_q) {
+          if (!mbar_wait(q_full + qb.idx, qb.phase, ctl, 12)) break;
+          if constexpr (kFP8) {
+            for (int s = 0; s < nsub; ++s) {
+              uint8_t *sf = sqsf + (qb.idx * kNSUB + s) * L.q_sf_bytes;
+              const int r = ((q.t0 + s * p.tq_sub) * p.H) & (kSfPad - 1);
+              for (int a = 0; a < atoms; ++a)
+                sf_reorder_atom(reinterpret_cast<const uint32_t *>(sf) + r + 128 * a,
+                                min(128, n_cols - 128 * a),
+                                reinterpret_cast<uint32_t *>(sf + sf_raw_bytes_q(n_cols) + 512 * a));
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tc_fence_after_sync();
+              for (int s = 0; s < nsub; ++s) {
+                uint8_t *sf = sqsf + (qb.idx * kNSUB + s) * L.q_sf_bytes;
+                for (int a = 0; a < atoms; ++a)
+                  tmem_cp_32x128b_x4(
+                      tmem_base + sfb_col0 + (qb.idx * kNSUB + s) * 4 * atoms + 4 * a,
+                      sdesc_rows16_noswizzle(smem_u32(sf + sf_raw_bytes_q(n_cols) + 512 * a)));
+              }
+            }
+          }
+          tc_fence_after_sync();
+          new_q = false;
+        }
+        if (!mbar_wait(full_k + st.idx, st.phase, ctl, 13)) break;
+        if constexpr (kFP8) {
+          uint8_t *sf = sksf + st.idx * L.k_sf_bytes;
+          const int r = (q.y0 + j * kBlockM) & (kSfPad - 1);
+          sf_reorder_atom(reinterpret_cast<const uint32_t *>(sf) + r, 128,
+                          reinterpret_cast<uint32_t *>(sf + kSfRawBytesK));
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tc_fence_after_sync();
+            tmem_cp_32x128b_x4(tmem_base + sfa_col0 + st.idx * 4,
+                               sdesc_rows16_noswizzle(smem_u32(sf + kSfRawBytesK)));
+          }
+        }
         tc_fence_after_sync();
+        const uint32_t k_base = smem_u32(sk + st.idx * L.k_stage_bytes);
         const uint32_t q_base = smem_u32(sq + qb.idx * kNSUB * L.q_sub_bytes);
         bool ok = true;
-        for (int j = U.j0; j < U.j_act && ok; ++j) {
-          if (!mbar_wait(full_k + st.idx, st.phase, ctl, 13)) { ok = false; break; }
+        for (int s = 0; s < nsub; ++s) {
+          if (!mbar_wait(acc_empty + ac.idx, ac.phase ^ 1u, ctl, 14)) { ok = false; break; }
           tc_fence_after_sync();
-          const uint32_t k_base = smem_u32(sk + st.idx * L.k_stage_bytes);
-          for (int s = 0; s < nsub; ++s) {
-            if (!mbar_wait(acc_empty + ac.idx, ac.phase ^ 1u, ctl, 14)) { ok = false; break; }
-            tc_fence_after_sync();
+          if (lane == 0) {
             const uint32_t d_tmem = tmem_base + ac.idx * n_cols;
             const uint32_t qs = q_base + s * L.q_sub_bytes;
+            if constexpr (kFP8) {
+              const uint32_t sfa = tmem_base + sfa_col0 + st.idx * 4;
+              const uint32_t sfb = tmem_base + sfb_col0 + (qb.idx * kNSUB + s) * 4 * atoms;
 #pragma unroll
-            for (int kk = 0; kk < kHeadDim / 16; ++kk) {
-              const uint32_t half = kk / 4, koff = (kk % 4) * 32;
-              const uint64_t ad = sdesc_kmajor_sw128(k_base + half * (kBlockM * 128) + koff);
-              const uint64_t bd = sdesc_kmajor_sw128(qs + half * (n_cols * 128) + koff);
-              mma_f16_ss(d_tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
+              for (int kk = 0; kk < kHeadDim / 32; ++kk) {
+                const uint64_t ad = sdesc_kmajor_sw128(k_base + kk * 32);
+                const uint64_t bd = sdesc_kmajor_sw128(qs + kk * 32);
+                mma_mxf8_ss(d_tmem, ad, bd, idesc_mxf8_e4m3(kBlockM, n_cols, kk, kk), sfa, sfb,
+                            kk > 0 ? 1u : 0u);
+              }
+            } else {
+              const uint32_t idesc = idesc_bf16_f32(kBlockM, n_cols);
+#pragma unroll
+              for (int kk = 0; kk < kHeadDim / 16; ++kk) {
+                const uint32_t half = kk / 4, koff = (kk % 4) * 32;
+                const uint64_t ad = sdesc_kmajor_sw128(k_base + half * (kBlockM * 128) + koff);
+                const uint64_t bd = sdesc_kmajor_sw128(qs + half * (n_cols * 128) + koff);
+                mma_f16_ss(d_tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
+              }
             }
             mma_commit(acc_full + ac.idx);
             last_commit = acc_full + ac.idx;
             last_commit_phase = ac.phase;
-            ac.next(kNACC);
           }
-          if (!ok) break;
-          mma_commit(empty_k + st.idx);      // stage free once these MMAs finish
-          st.next(kSTAGES);
+          __syncwarp();
+          ac.next(kNACC);
         }
         if (!ok) break;
-        mma_commit(q_empty + qb.idx);
-        qb.next(kQBUF);
+        if (lane == 0) mma_commit(empty_k + st.idx);   // stage free once these MMAs finish
+        __syncwarp();
+        st.next(kSTAGES);
+        bool block_done = n + 1 == R.a_count;
+        if (!block_done) {
+          const int pb = q.b, ps = q.seq;
+          next_active(p, tqt, q, j);
+          block_done = q.b != pb || q.seq != ps;
+        }
+        if (block_done) {
+          if (lane == 0) mma_commit(q_empty + qb.idx);
+          __syncwarp();
+          qb.next(kQBUF);
+          new_q = true;
+        }
       }
       // MMAs still in flight must finish before TMEM is released.
-      if (last_commit) mbar_drain(last_commit, last_commit_phase, p.wait_limit_ns);
+      if (lane == 0 && last_commit) mbar_drain(last_commit, last_commit_phase, p.wait_limit_ns);
+      __syncwarp();
     }
   } else {
     // ---------------- epilogue ----------------
@@ -351,45 +680,47 @@ __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
     const int quad = warp & 3;                 // TMEM lane quadrant of this warp
     const int group = epi / 4;                 // token subset of this warp
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
-    Ring ac, sc;
-    for (;;) {
-      if (!mbar_wait(sched_full + sc.idx, sc.phase, ctl, 21)) break;
-      const uint32_t u = sched_unit[sc.idx];
-      __syncwarp();
-      if (lane == 0) mbar_arrive(sched_empty + sc.idx);
-      sc.next(kSchedSlots);
-      Unit U;
-      if (!decode_unit(p, tq_total, u, U)) break;
-      const int nsub = (U.ntok + p.tq_sub - 1) / p.tq_sub;
-      bool ok = true;
-      for (int j = U.j0; j < U.j1 && ok; ++j) {
+    // Fully masked tiles first: plain stores while the first loads are in flight.
+    if (R.f_count > 0) {
+      QBlk q;
+      int j = R.f_j;
+      make_qb(p, tqt, R.f_seq, R.f_b, R.f_seqoff, q);
+      for (int64_t n = 0; n < R.f_count; ++n) {
         const int64_t slot = static_cast<int64_t>(j) * kBlockM + quad * 32 + lane;
-        const bool in_row = slot < U.row_len;
-        if (j >= U.j_act) {
-          // every token of the unit is masked on this whole tile
-          if (in_row)
-            for (int i = group; i < U.ntok; i += kGroups)
-              p.scores[U.out0 + i * U.row_len + slot] = kMaskBound;
-          continue;
-        }
+        if (slot < q.row_len)
+          for (int i = group; i < q.ntok; i += kGroups)
+            p.scores[q.out0 + i * q.row_len + slot] = kMaskBound;
+        if (n + 1 < R.f_count) next_fill(p, tqt, q, j);
+      }
+    }
+    if (R.a_count > 0) {
+      Ring ac;
+      QBlk q;
+      int j = R.a_j;
+      make_qb(p, tqt, R.a_seq, R.a_b, R.a_seqoff, q);
+      bool ok = true;
+      for (int64_t n = 0; n < R.a_count && ok; ++n) {
+        const int nsub = (q.ntok + p.tq_sub - 1) / p.tq_sub;
+        const int64_t slot = static_cast<int64_t>(j) * kBlockM + quad * 32 + lane;
+        const bool in_row = slot < q.row_len;
         for (int s = 0; s < nsub; ++s) {
           if (!mbar_wait(acc_full + ac.idx, ac.phase, ctl, 22)) { ok = false; break; }
           tc_fence_after_sync();
           const uint32_t tbase = tmem_base + lane_addr + ac.idx * n_cols;
           const int i0 = s * p.tq_sub;
-          const int ntok_s = min(p.tq_sub, U.ntok - i0);
+          const int ntok_s = min(p.tq_sub, q.ntok - i0);
           if constexpr (kH == 64) {
             for (int i = group; i < ntok_s; i += kGroups) {
-              const int t = U.t0 + i0 + i;
+              const int t = q.t0 + i0 + i;
               const float acc = head_sum_h64(tbase + i * 64, p.w + static_cast<int64_t>(t) * 64);
-              const int lv = unit_last_valid(p, U, i0 + i);
+              const int lv = qb_last_valid(p, q, i0 + i);
               if (in_row)
-                p.scores[U.out0 + (i0 + i) * U.row_len + slot] = slot <= lv ? acc : kMaskBound;
+                p.scores[q.out0 + (i0 + i) * q.row_len + slot] = slot <= lv ? acc : kMaskBound;
             }
           } else {
             // any H: walk the sub-block's columns in 16-wide chunks
             const int H = p.H, ncols = ntok_s * H;
-            const float *wsub = p.w + static_cast<int64_t>(U.t0 + i0) * H;
+            const float *wsub = p.w + static_cast<int64_t>(q.t0 + i0) * H;
             float acc = 0.f;
             int tok = 0, h = 0;
             for (int c0 = 0; c0 < ncols; c0 += 16) {
@@ -400,11 +731,13 @@ __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
                 if (c0 + c < ncols) {
                   acc = fmaf(__ldg(wsub + c0 + c), fmaxf(v[c], 0.f), acc);
                   if (++h == H) {
-                    const int lv = unit_last_valid(p, U, i0 + tok);
+                    const int lv = qb_last_valid(p, q, i0 + tok);
                     if (in_row)
-                      p.scores[U.out0 + (i0 + tok) * U.row_len + slot] =
+                      p.scores[q.out0 + (i0 + tok) * q.row_len + slot] =
                           slot <= lv ? acc : kMaskBound;
-                    acc = 0.f; h = 0; ++tok;
+                    acc = 0.f;
+                    h = 0;
+                    ++tok;
                   }
                 }
               }
@@ -415,8 +748,8 @@ __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
           if (lane == 0) mbar_arrive(acc_empty + ac.idx);
           ac.next(kNACC);
         }
+        if (ok && n + 1 < R.a_count) next_active(p, tqt, q, j);
       }
-      if (!ok) break;
     }
   }
 
@@ -424,16 +757,6 @@ __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
   __syncthreads();
   tc_fence_after_sync();
   if (warp == 1) tmem_dealloc(tmem_base, tmem_cols);
-  // The last CTA to finish leaves the scheduler counters at zero for the
-  // next launch on this workspace (every fetch of this launch is done).
-  if (threadIdx.x == 0) {
-    __threadfence();
-    if (atomicAdd(p.done_counter, 1u) == gridDim.x - 1) {
-      atomicExch(p.sched_counter, 0u);
-      atomicExch(p.done_counter, 0u);
-      __threadfence();
-    }
-  }
 }
 
 }  // namespace dsa

@@ -123,6 +123,15 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
                : "memory");
 }
 
+__device__ __forceinline__ void tma_load_1d(void *dst, const CUtensorMap *map,
+                                            uint64_t *bar, int32_t c0) {
+  asm volatile(
+      "cp.async.bulk.tensor.1d.shared::cluster.global.tile.mbarrier::complete_"
+      "tx::bytes [%0], [%1, {%3}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0)
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map,
                                             uint64_t *bar, int32_t c0,
                                             int32_t c1) {
@@ -270,6 +279,68 @@ __device__ __forceinline__ void tmem_ld16_wait(uint32_t taddr, float (&v)[16]) {
       : "memory");
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+}  // namespace dsa
+
+namespace dsa {
+
+// ---- block-scaled fp8 (MX) MMA ------------------------------------------------
+
+// D[tmem] (+)= (A * sfA) * (B * sfB)^T with e4m3 A and B, ue8m0 scale
+// factors per 32 elements of K read from TMEM, fp32 accumulate.
+__device__ __forceinline__ void mma_mxf8_ss(uint32_t tmem_d, uint64_t adesc,
+                                            uint64_t bdesc, uint32_t idesc,
+                                            uint32_t tmem_sfa, uint32_t tmem_sfb,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, "
+      "[%5], [%6], p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tmem_sfa),
+      "r"(tmem_sfb)
+      : "memory");
+}
+
+// Instruction descriptor of kind::mxf8f6f4 with block scaling: e4m3 A and B,
+// both K-major, ue8m0 scales; sf_a / sf_b pick the scale byte (K block of 32)
+// inside each 32-bit TMEM scale word.
+__host__ __device__ constexpr uint32_t idesc_mxf8_e4m3(uint32_t M, uint32_t N,
+                                                       uint32_t sf_a,
+                                                       uint32_t sf_b) {
+  return (sf_b << 4)          // B scale-factor byte
+         | (0u << 7)          // A format: e4m3
+         | (0u << 10)         // B format: e4m3
+         | ((N >> 3) << 17)   // N / 8
+         | (1u << 23)         // scale format: ue8m0
+         | ((M >> 4) << 24)   // M / 16
+         | (sf_a << 29);      // A scale-factor byte
+}
+
+// Shared-memory source of tcgen05.cp.32x128b: 32 rows of 16 bytes stored
+// contiguously (no swizzle, K-major core matrices of 8 rows x 16 bytes).
+__device__ __forceinline__ uint64_t sdesc_rows16_noswizzle(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);       // start address
+  d |= static_cast<uint64_t>(128u >> 4) << 16;              // LBO
+  d |= static_cast<uint64_t>(128u >> 4) << 32;              // SBO: 8 rows
+  d |= static_cast<uint64_t>(1u) << 46;                     // sm100 version
+  return d;                                                 // layout 0: none
+}
+
+// Copy 32 rows x 128 bits from shared memory into TMEM lanes 0..31 of each
+// of the four lane quadrants (4 columns of 32 bits).
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr),
+               "l"(sdesc)
+               : "memory");
+}
+
+// Make generic-proxy writes to shared memory visible to the async proxy
+// (TMA, tcgen05.cp, tcgen05.mma operand reads).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 }  // namespace dsa

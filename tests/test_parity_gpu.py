@@ -130,3 +130,55 @@ def test_ragged_prefill_full_size_sampled(dsa):
         rows += [cu[i], cu[i] + 1, cu[i] + 2049, cu[i + 1] - 1]
     rows += list(rng.integers(0, wl.T, 8))
     run_and_check(dsa, wl, syn.generate(wl), rows=sorted(set(int(r) for r in rows)))
+
+
+# ---- fp8 e4m3 + block-32 e8m0 (block-scaled MMA) -------------------------------
+
+from parity_util import TOL_FP8  # noqa: E402
+
+
+def fp8_decode_wl(T=3, H=64, S=700, k=50, shared=False, pos=(0, 700), seed=0):
+    return syn.Workload("d8", syn.MODE_POSITIONS, T=T, H=H, D=128, index_topk=k,
+                        S=S, shared_cache=shared, pos_lo=pos[0], pos_hi=pos[1],
+                        dtype=syn.DTYPE_FP8, w_scale=1.0 / np.sqrt(H), seed=seed)
+
+
+def fp8_causal_wl(seqlens, H=64, k=64, seed=0):
+    return syn.Workload("c8", syn.MODE_CAUSAL, T=int(sum(seqlens)), H=H, D=128,
+                        index_topk=k, seqlens=tuple(seqlens), dtype=syn.DTYPE_FP8,
+                        w_scale=1.0 / np.sqrt(H), seed=seed)
+
+
+@pytest.mark.parametrize("H", [4, 16, 64, 128])
+def test_fp8_decode_heads(dsa, H):
+    wl = fp8_decode_wl(T=3, H=H, S=700, k=100, seed=20 + H)
+    run_and_check(dsa, wl, syn.generate(wl), tol=TOL_FP8)
+
+
+@pytest.mark.parametrize("H", [4, 64])
+def test_fp8_integer_inputs_bit_exact(dsa, H):
+    wl = fp8_decode_wl(T=3, H=H, S=520, k=32, pos=(100, 520), seed=5)
+    run_and_check(dsa, wl, syn.generate(wl, value_kind="int"), tol=TOL_FP8, exact=True)
+
+
+@pytest.mark.parametrize("H", [4, 64])
+def test_fp8_causal_ragged(dsa, H):
+    wl = fp8_causal_wl((1, 127, 129, 300, 1000), H=H, k=64, seed=30 + H)
+    run_and_check(dsa, wl, syn.generate(wl), tol=TOL_FP8)
+
+
+def test_fp8_causal_integer_bit_exact(dsa):
+    wl = fp8_causal_wl((130, 257), H=64, k=16, seed=6)
+    run_and_check(dsa, wl, syn.generate(wl, value_kind="int"), tol=TOL_FP8, exact=True)
+
+
+def test_fp8_shared_cache(dsa):
+    wl = fp8_decode_wl(T=9, H=64, S=900, k=50, shared=True, seed=7)
+    run_and_check(dsa, wl, syn.generate(wl), tol=TOL_FP8)
+
+
+def test_long_decode_fp8_full_size_sampled(dsa):
+    wl = syn.WORKLOADS["long_decode_fp8"]
+    rng = np.random.default_rng(13)
+    rows = sorted(set([0, 1, 63] + list(rng.integers(0, wl.T, 5))))
+    run_and_check(dsa, wl, syn.generate(wl), rows=rows, tol=TOL_FP8)

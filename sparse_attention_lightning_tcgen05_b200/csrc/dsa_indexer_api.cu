@@ -278,9 +278,6 @@ dsa_status_t launch_topk(const dsa_indexer_desc_t *d, const float *scores,
   DeviceInfo *dev = nullptr;
   dsa_status_t st = device_info(&dev);
   if (st != DSA_OK) return st;
-  const int smem = static_cast<int>(sizeof(dsa::TopkSmem));
-  st = ensure_smem_attr(dev, 8, dsa::topk_kernel, smem);
-  if (st != DSA_OK) return st;
   TopkParams p{};
   p.mode = d->mask == DSA_MASK_CAUSAL ? dsa::kModeCausal : dsa::kModePositions;
   p.T = d->T;
@@ -291,7 +288,25 @@ dsa_status_t launch_topk(const dsa_indexer_desc_t *d, const float *scores,
   p.scores = scores;
   p.topk = topk;
   p.k = d->index_topk;
-  dsa::topk_kernel<<<d->T, dsa::kTopkThreads, smem, stream>>>(p);
+  // Decode rows are few and long: 1024 threads a row, the row staged in
+  // shared memory when it fits. Prefill rows are many: 512 threads a row and
+  // a smaller stage, so that several rows run on each SM.
+  if (p.mode == dsa::kModePositions) {
+    using Sh = dsa::TopkShared<1024>;
+    const int64_t room = (kMaxSmemPerBlock - sizeof(Sh) - 1024) / 4;
+    p.stage_cap = static_cast<int>(std::min<int64_t>(d->S, room));
+    const int smem = static_cast<int>(sizeof(Sh) + 4 * static_cast<size_t>(p.stage_cap));
+    st = ensure_smem_attr(dev, 8, dsa::topk_kernel<1024>, static_cast<int>(kMaxSmemPerBlock));
+    if (st != DSA_OK) return st;
+    dsa::topk_kernel<1024><<<d->T, 1024, smem, stream>>>(p);
+  } else {
+    using Sh = dsa::TopkShared<512>;
+    p.stage_cap = std::min(d->T, 12288);
+    const int smem = static_cast<int>(sizeof(Sh) + 4 * static_cast<size_t>(p.stage_cap));
+    st = ensure_smem_attr(dev, 9, dsa::topk_kernel<512>, static_cast<int>(kMaxSmemPerBlock));
+    if (st != DSA_OK) return st;
+    dsa::topk_kernel<512><<<d->T, 512, smem, stream>>>(p);
+  }
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 

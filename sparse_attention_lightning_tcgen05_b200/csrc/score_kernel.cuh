@@ -83,10 +83,14 @@ __host__ __device__ constexpr uint32_t sf_raw_bytes_q(int n_cols) {
 }
 
 // Shared-memory plan, identical on host and device.
+constexpr int kPosCap = 2048;          // positions staged in shared memory
+constexpr int kWRowsPerWarp = 4;        // H=64 epilogue: w rows a warp keeps
+
 struct ScoreSmem {
   uint32_t k_stage_bytes, k_sf_bytes, q_sub_bytes, q_sf_bytes;
-  uint32_t off_k, off_ksf, off_q, off_qsf, off_bar, off_misc, total;
-  __host__ __device__ ScoreSmem(int stages, int qbuf, int nsub, int n_cols, bool fp8) {
+  uint32_t off_k, off_ksf, off_q, off_qsf, off_w, off_pos, off_bar, off_misc, total;
+  __host__ __device__ ScoreSmem(int stages, int qbuf, int nsub, int n_cols, bool fp8,
+                                int epi_warps = 8) {
     // bf16: two 128-byte-wide halves along D; fp8: one 128-byte row.
     k_stage_bytes = fp8 ? kBlockM * 128 : kBlockM * 256;
     q_sub_bytes = fp8 ? n_cols * 128 : n_cols * 256;
@@ -99,8 +103,10 @@ struct ScoreSmem {
     off_q = off_k + stages * k_stage_bytes;
     off_ksf = off_q + qbuf * nsub * q_sub_bytes;
     off_qsf = off_ksf + stages * k_sf_bytes;
-    off_bar = off_qsf + qbuf * nsub * q_sf_bytes;
-    off_bar = (off_bar + 15) & ~15u;
+    off_w = off_qsf + qbuf * nsub * q_sf_bytes;
+    off_w = (off_w + 15) & ~15u;
+    off_pos = off_w + epi_warps * kWRowsPerWarp * 64 * 4;
+    off_bar = off_pos + kPosCap * 4;
     off_misc = off_bar + 64 * 8;            // up to 64 mbarriers
     total = off_misc + 256 + 1024;          // misc words + alignment slack
   }
@@ -128,7 +134,7 @@ struct QBlk {
 };
 
 __device__ __forceinline__ int last_valid_pos(const ScoreParams &p, int t) {
-  const int pos = __ldg(p.positions + t);
+  const int pos = p.positions[t];     // global, or the CTA's shared copy
   const int64_t lv = pos < 0 ? -1 : (pos >= p.S ? p.S - 1 : pos);
   return static_cast<int>(lv);
 }
@@ -142,7 +148,7 @@ __device__ __forceinline__ int pos_num_blocks(const ScoreParams &p, int tqt) {
   return p.shared_cache ? (p.T + tqt - 1) / tqt : p.T;
 }
 
-__device__ void make_qb_positions(const ScoreParams &p, int tqt, int b, QBlk &q) {
+__device__ __forceinline__ void make_qb_positions(const ScoreParams &p, int tqt, int b, QBlk &q) {
   q.seq = 0;
   q.b = b;
   q.t0 = b * tqt;
@@ -159,7 +165,7 @@ __device__ void make_qb_positions(const ScoreParams &p, int tqt, int b, QBlk &q)
   q.act = mx < 0 ? 0 : mx / kBlockM + 1;
 }
 
-__device__ void make_qb_causal(const ScoreParams &p, int tqt, int seq, int b,
+__device__ __forceinline__ void make_qb_causal(const ScoreParams &p, int tqt, int seq, int b,
                                int64_t seqoff, QBlk &q) {
   const int a = __ldg(p.cu_seqlens + seq);
   const int L = __ldg(p.cu_seqlens + seq + 1) - a;
@@ -187,7 +193,7 @@ __device__ __forceinline__ int64_t causal_active_before(int64_t B, int r) {
 }
 
 // Move q to the next query block (skipping empty sequences). False at the end.
-__device__ bool next_qb(const ScoreParams &p, int tqt, QBlk &q) {
+__device__ __forceinline__ bool next_qb(const ScoreParams &p, int tqt, QBlk &q) {
   if (p.mode == kModePositions) {
     if (q.b + 1 >= pos_num_blocks(p, tqt)) return false;
     make_qb_positions(p, tqt, q.b + 1, q);
@@ -231,7 +237,7 @@ __device__ __forceinline__ int64_t warp_incl_scan64(int64_t v) {
 
 // POSITIONS: the block holding item `idx` of the active (fill == false) or
 // fill list, by a warp-wide scan over blocks. Executed by a full warp.
-__device__ void locate_positions(const ScoreParams &p, int tqt, int64_t idx, bool fill,
+__device__ __forceinline__ void locate_positions(const ScoreParams &p, int tqt, int64_t idx, bool fill,
                                  int &b_out, int &j_out) {
   const int lane = threadIdx.x & 31;
   const int nqb = pos_num_blocks(p, tqt);
@@ -264,7 +270,7 @@ __device__ void locate_positions(const ScoreParams &p, int tqt, int64_t idx, boo
 }
 
 // POSITIONS: total active and fill items (full warp).
-__device__ void count_positions(const ScoreParams &p, int tqt, int64_t &A, int64_t &F) {
+__device__ __forceinline__ void count_positions(const ScoreParams &p, int tqt, int64_t &A, int64_t &F) {
   const int lane = threadIdx.x & 31;
   const int nqb = pos_num_blocks(p, tqt);
   int64_t a = 0, f = 0;
@@ -290,7 +296,7 @@ __device__ __forceinline__ int64_t causal_before(int64_t B, int r, int ntr, bool
 }
 
 // CAUSAL: locate item idx of the active or fill list (one thread).
-__device__ void locate_causal(const ScoreParams &p, int tqt, int64_t idx, bool fill,
+__device__ __forceinline__ void locate_causal(const ScoreParams &p, int tqt, int64_t idx, bool fill,
                               int &seq_out, int &b_out, int &j_out, int64_t &seqoff_out) {
   const int r = kBlockM / tqt;
   int64_t off = 0;
@@ -320,7 +326,7 @@ __device__ void locate_causal(const ScoreParams &p, int tqt, int64_t idx, bool f
   seqoff_out = off;
 }
 
-__device__ void count_causal(const ScoreParams &p, int tqt, int64_t &A, int64_t &F) {
+__device__ __forceinline__ void count_causal(const ScoreParams &p, int tqt, int64_t &A, int64_t &F) {
   const int r = kBlockM / tqt;
   A = 0;
   F = 0;
@@ -335,7 +341,7 @@ __device__ void count_causal(const ScoreParams &p, int tqt, int64_t &A, int64_t 
 
 // This CTA's share of both lists (executed by a full warp; every lane gets
 // the same result).
-__device__ void cta_range(const ScoreParams &p, int tqt, CtaRange &R) {
+__device__ __forceinline__ void cta_range(const ScoreParams &p, int tqt, CtaRange &R) {
   const int64_t G = gridDim.x, c = blockIdx.x;
   int64_t A = 0, F = 0;
   if (p.mode == kModePositions) count_positions(p, tqt, A, F);
@@ -386,25 +392,42 @@ __device__ __forceinline__ bool next_fill(const ScoreParams &p, int tqt, QBlk &q
 
 // ---- epilogue helpers ---------------------------------------------------------------
 
-// One token with H == 64 (the tuned head count): the two 32-column TMEM
-// loads hold heads 0..31 and 32..63 of this slot.
+// One token with H == 64 (the tuned head count): one load of the 64 TMEM
+// columns (heads 0..63 of this slot), w row from shared memory, four
+// independent partial sums.
 __device__ __forceinline__ float head_sum_h64(uint32_t taddr, const float *wrow) {
-  float v[32];
-  float acc = 0.f;
+  uint32_t r[64];
+  tmem_ld64_wait(taddr, r);
   const float4 *w4 = reinterpret_cast<const float4 *>(wrow);
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    tmem_ld32_wait(taddr + half * 32, v);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float4 wv = __ldg(w4 + half * 8 + i);
-      acc = fmaf(wv.x, fmaxf(v[4 * i + 0], 0.f), acc);
-      acc = fmaf(wv.y, fmaxf(v[4 * i + 1], 0.f), acc);
-      acc = fmaf(wv.z, fmaxf(v[4 * i + 2], 0.f), acc);
-      acc = fmaf(wv.w, fmaxf(v[4 * i + 3], 0.f), acc);
-    }
+  for (int i = 0; i < 16; ++i) {
+    const float4 wv = w4[i];
+    a0 = fmaf(wv.x, fmaxf(__uint_as_float(r[4 * i + 0]), 0.f), a0);
+    a1 = fmaf(wv.y, fmaxf(__uint_as_float(r[4 * i + 1]), 0.f), a1);
+    a2 = fmaf(wv.z, fmaxf(__uint_as_float(r[4 * i + 2]), 0.f), a2);
+    a3 = fmaf(wv.w, fmaxf(__uint_as_float(r[4 * i + 3]), 0.f), a3);
   }
-  return acc;
+  return (a0 + a1) + (a2 + a3);
+}
+
+__device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+
+// Write the mask bound to row[lo, hi), threads t = 0..nthr-1 of the caller,
+// 16-byte stores on the aligned body.
+__device__ __forceinline__ void fill_mask(float *row, int64_t lo, int64_t hi, int t, int nthr) {
+  if (lo >= hi) return;
+  float *base = row + lo;
+  const int64_t n = hi - lo;
+  const int64_t head =
+      min64(n, ((16 - (reinterpret_cast<uintptr_t>(base) & 15)) & 15) / 4);
+  if (t < head) base[t] = kMaskBound;
+  const int64_t nvec = (n - head) / 4;
+  float4 *v = reinterpret_cast<float4 *>(base + head);
+  const float4 mb = make_float4(kMaskBound, kMaskBound, kMaskBound, kMaskBound);
+  for (int64_t i = t; i < nvec; i += nthr) v[i] = mb;
+  const int64_t tail0 = head + 4 * nvec;
+  if (tail0 + t < n) base[tail0 + t] = kMaskBound;
 }
 
 // Role bookkeeping of a ring of mbarrier pairs.
@@ -448,7 +471,7 @@ __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const ScoreSmem L(kSTAGES, kQBUF, kNSUB, p.n_cols, kFP8);
+  const ScoreSmem L(kSTAGES, kQBUF, kNSUB, p.n_cols, kFP8, kEPI);
   uint8_t *sk = smem + L.off_k;
   uint8_t *sq = smem + L.off_q;
   uint8_t *sksf = smem + L.off_ksf;
@@ -475,9 +498,18 @@ __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
                          tmem_cols_needed(kNACC, n_cols, kSTAGES, kQBUF, kNSUB, kFP8)))
     tmem_cols <<= 1;
 
+  // Decode positions are read by every role many times: keep a copy here.
+  int *spos = reinterpret_cast<int *>(smem + L.off_pos);
+  const bool pos_staged = p.mode == kModePositions && p.T <= kPosCap;
+  if (pos_staged)
+    for (int i = threadIdx.x; i < p.T; i += blockDim.x) spos[i] = __ldg(p.positions + i);
+  __syncthreads();
+  ScoreParams P = p;
+  if (pos_staged) P.positions = spos;
+
   if (warp == 0) {
     CtaRange R;
-    cta_range(p, tqt, R);
+    cta_range(P, tqt, R);
     if (lane == 0) {
       *range_slot = R;
       for (int i = 0; i < kSTAGES; ++i) { mbar_init(full_k + i, 1); mbar_init(empty_k + i, 1); }
@@ -512,7 +544,7 @@ __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
       uint32_t k_issued = 0, q_issued = 0, k_last_phase = 0, q_last_phase = 0;
       QBlk q;
       int j = R.a_j;
-      make_qb(p, tqt, R.a_seq, R.a_b, R.a_seqoff, q);
+      make_qb(P, tqt, R.a_seq, R.a_b, R.a_seqoff, q);
       bool need_q = true;
       for (int64_t n = 0; n < R.a_count; ++n) {
         if (need_q) {
@@ -553,7 +585,7 @@ __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
         st.next(kSTAGES);
         if (n + 1 < R.a_count) {
           const int pb = q.b, ps = q.seq;
-          next_active(p, tqt, q, j);
+          next_active(P, tqt, q, j);
           if (q.b != pb || q.seq != ps) { need_q = true; qb.next(kQBUF); }
         }
       }
@@ -571,7 +603,7 @@ __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
       uint32_t last_commit_phase = 0;
       QBlk q;
       int j = R.a_j;
-      make_qb(p, tqt, R.a_seq, R.a_b, R.a_seqoff, q);
+      make_qb(P, tqt, R.a_seq, R.a_b, R.a_seqoff, q);
       bool new_q = true;
       for (int64_t n = 0; n < R.a_count; ++n) {
         const int nsub = (q.ntok + p.tq_sub - 1) / p.tq_sub;
@@ -660,7 +692,7 @@ __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
         bool block_done = n + 1 == R.a_count;
         if (!block_done) {
           const int pb = q.b, ps = q.seq;
-          next_active(p, tqt, q, j);
+          next_active(P, tqt, q, j);
           block_done = q.b != pb || q.seq != ps;
         }
         if (block_done) {
@@ -680,27 +712,60 @@ __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
     const int quad = warp & 3;                 // TMEM lane quadrant of this warp
     const int group = epi / 4;                 // token subset of this warp
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
-    // Fully masked tiles first: plain stores while the first loads are in flight.
+    // Fully masked tiles first, while the first loads are in flight: each run
+    // of masked tiles of a query block is one contiguous slot range per
+    // token, written by all epilogue threads with 16-byte stores.
     if (R.f_count > 0) {
       QBlk q;
       int j = R.f_j;
-      make_qb(p, tqt, R.f_seq, R.f_b, R.f_seqoff, q);
-      for (int64_t n = 0; n < R.f_count; ++n) {
-        const int64_t slot = static_cast<int64_t>(j) * kBlockM + quad * 32 + lane;
-        if (slot < q.row_len)
-          for (int i = group; i < q.ntok; i += kGroups)
-            p.scores[q.out0 + i * q.row_len + slot] = kMaskBound;
-        if (n + 1 < R.f_count) next_fill(p, tqt, q, j);
+      make_qb(P, tqt, R.f_seq, R.f_b, R.f_seqoff, q);
+      const int et = epi * 32 + lane;
+      int64_t left = R.f_count;
+      while (left > 0) {
+        const int64_t seg = min64(left, q.ntr - j);
+        const int64_t lo = static_cast<int64_t>(j) * kBlockM;
+        const int64_t hi = min64(static_cast<int64_t>(j + seg) * kBlockM, q.row_len);
+        for (int i = 0; i < q.ntok; ++i)
+          fill_mask(p.scores + q.out0 + i * q.row_len, lo, hi, et, kEPI * 32);
+        left -= seg;
+        if (left > 0) {
+          do {
+            if (!next_qb(P, tqt, q)) { left = 0; break; }
+          } while (q.act == q.ntr);
+          j = q.act;
+        }
       }
     }
     if (R.a_count > 0) {
       Ring ac;
       QBlk q;
       int j = R.a_j;
-      make_qb(p, tqt, R.a_seq, R.a_b, R.a_seqoff, q);
+      make_qb(P, tqt, R.a_seq, R.a_b, R.a_seqoff, q);
       bool ok = true;
+      // H=64: this warp's w rows for the current query block (warp-private)
+      float *wrows = reinterpret_cast<float *>(smem + L.off_w) + epi * kWRowsPerWarp * 64;
+      int w_seq = -1, w_b = -1;
       for (int64_t n = 0; n < R.a_count && ok; ++n) {
         const int nsub = (q.ntok + p.tq_sub - 1) / p.tq_sub;
+        if constexpr (kH == 64) {
+          if (q.b != w_b || q.seq != w_seq) {
+            w_b = q.b;
+            w_seq = q.seq;
+            const int per = (p.tq_sub + kGroups - 1) / kGroups;
+            __syncwarp();
+            for (int s = 0; s < nsub; ++s) {
+              const int ntok_s = min(p.tq_sub, q.ntok - s * p.tq_sub);
+              const int i_lo = min(ntok_s, group * per), i_hi = min(ntok_s, i_lo + per);
+              for (int idx = lane; idx < (i_hi - i_lo) * 16; idx += 32) {
+                const int u = idx / 16, c = idx % 16;
+                const int t = q.t0 + s * p.tq_sub + i_lo + u;
+                reinterpret_cast<float4 *>(wrows + (s * per + u) * 64)[c] =
+                    __ldg(reinterpret_cast<const float4 *>(p.w + static_cast<int64_t>(t) * 64) + c);
+              }
+            }
+            __syncwarp();
+          }
+        }
         const int64_t slot = static_cast<int64_t>(j) * kBlockM + quad * 32 + lane;
         const bool in_row = slot < q.row_len;
         for (int s = 0; s < nsub; ++s) {
@@ -710,12 +775,17 @@ __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
           const int i0 = s * p.tq_sub;
           const int ntok_s = min(p.tq_sub, q.ntok - i0);
           if constexpr (kH == 64) {
-            for (int i = group; i < ntok_s; i += kGroups) {
-              const int t = q.t0 + i0 + i;
-              const float acc = head_sum_h64(tbase + i * 64, p.w + static_cast<int64_t>(t) * 64);
-              const int lv = qb_last_valid(p, q, i0 + i);
-              if (in_row)
-                p.scores[q.out0 + (i0 + i) * q.row_len + slot] = slot <= lv ? acc : kMaskBound;
+            // this warp's tokens of the sub-block: adjacent pair (or one)
+            const int per = (p.tq_sub + kGroups - 1) / kGroups;
+            const int i_lo = min(ntok_s, group * per), i_hi = min(ntok_s, i_lo + per);
+            const float *wsh = wrows + (s * per) * 64;
+            {
+              for (int i = i_lo; i < i_hi; ++i) {
+                const float acc = head_sum_h64(tbase + i * 64, wsh + (i - i_lo) * 64);
+                const int lv = qb_last_valid(P, q, i0 + i);
+                if (in_row)
+                  p.scores[q.out0 + (i0 + i) * q.row_len + slot] = slot <= lv ? acc : kMaskBound;
+              }
             }
           } else {
             // any H: walk the sub-block's columns in 16-wide chunks
@@ -731,7 +801,7 @@ __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
                 if (c0 + c < ncols) {
                   acc = fmaf(__ldg(wsub + c0 + c), fmaxf(v[c], 0.f), acc);
                   if (++h == H) {
-                    const int lv = qb_last_valid(p, q, i0 + tok);
+                    const int lv = qb_last_valid(P, q, i0 + tok);
                     if (in_row)
                       p.scores[q.out0 + (i0 + tok) * q.row_len + slot] =
                           slot <= lv ? acc : kMaskBound;
@@ -748,7 +818,7 @@ __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
           if (lane == 0) mbar_arrive(acc_empty + ac.idx);
           ac.next(kNACC);
         }
-        if (ok && n + 1 < R.a_count) next_active(p, tqt, q, j);
+        if (ok && n + 1 < R.a_count) next_active(P, tqt, q, j);
       }
     }
   }

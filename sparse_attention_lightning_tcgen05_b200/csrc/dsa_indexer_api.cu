@@ -9,10 +9,12 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "dsa_indexer.h"
 #include "dsa_launch.h"
 #include "score_kernel.cuh"
+#include "topk_cluster.cuh"
 #include "topk_kernel.cuh"
 
 namespace dsa_host {
@@ -148,6 +150,33 @@ struct ScoreLaunch {
   bool fp8;
 };
 
+// Launch with programmatic stream serialisation: the kernel may start while
+// the previous kernel on the stream is finishing; each kernel calls
+// griddepcontrol.wait before it touches memory that earlier work wrote.
+// `cluster` > 0 launches thread-block clusters of that many CTAs along x.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int threads, size_t smem,
+                       cudaStream_t stream, int cluster, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(static_cast<unsigned>(threads));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cluster > 0) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = static_cast<unsigned>(cluster);
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+  }
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 int round16(int x) { return (x + 15) / 16 * 16; }
 
 // Largest power of two <= x (x >= 1).
@@ -269,7 +298,9 @@ dsa_status_t launch_score(const dsa_indexer_desc_t *d, const void *q, const uint
     const int64_t nqb = p.shared_cache ? (d->T + tqt - 1) / tqt : d->T;
     if (nqb * ntiles < grid) grid = static_cast<int>(nqb * ntiles);
   }
-  L.kernel<<<grid, L.threads, plan.total, stream>>>(tk, tq, tksf, tqsf, p);
+  if (launch_pdl(L.kernel, grid, L.threads, plan.total, stream, 0, tk, tq, tksf, tqsf, p) !=
+      cudaSuccess)
+    return DSA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
@@ -288,24 +319,31 @@ dsa_status_t launch_topk(const dsa_indexer_desc_t *d, const float *scores,
   p.scores = scores;
   p.topk = topk;
   p.k = d->index_topk;
-  // Decode rows are few and long: 1024 threads a row, the row staged in
-  // shared memory when it fits. Prefill rows are many: 512 threads a row and
-  // a smaller stage, so that several rows run on each SM.
+  // Decode rows are few and long: a cluster of C CTAs per row (up to 8, about
+  // 4096 slots each), the row staged across their shared memories. Prefill
+  // rows are many: 512 threads a row and a smaller stage, so that several
+  // rows run on each SM.
   if (p.mode == dsa::kModePositions) {
-    using Sh = dsa::TopkShared<1024>;
+    using Sh = dsa::ClusterTopkShared<512>;
+    const int C = static_cast<int>(std::min<int64_t>(dsa::kClusterMaxRanks,
+                                                     std::max<int64_t>(1, (d->S + 4095) / 4096)));
+    if (static_cast<int64_t>(d->T) * C > INT32_MAX) return DSA_ERR_UNSUPPORTED;
     const int64_t room = (kMaxSmemPerBlock - sizeof(Sh) - 1024) / 4;
-    p.stage_cap = static_cast<int>(std::min<int64_t>(d->S, room));
+    p.stage_cap = static_cast<int>(std::min<int64_t>((d->S + C - 1) / C, room));
     const int smem = static_cast<int>(sizeof(Sh) + 4 * static_cast<size_t>(p.stage_cap));
-    st = ensure_smem_attr(dev, 8, dsa::topk_kernel<1024>, static_cast<int>(kMaxSmemPerBlock));
+    st = ensure_smem_attr(dev, 8, dsa::topk_cluster_kernel<512>, static_cast<int>(kMaxSmemPerBlock));
     if (st != DSA_OK) return st;
-    dsa::topk_kernel<1024><<<d->T, 1024, smem, stream>>>(p);
+    if (launch_pdl(dsa::topk_cluster_kernel<512>, d->T * C, 512, smem, stream, C, p) !=
+        cudaSuccess)
+      return DSA_ERR_CUDA;
   } else {
     using Sh = dsa::TopkShared<512>;
     p.stage_cap = std::min(d->T, 12288);
     const int smem = static_cast<int>(sizeof(Sh) + 4 * static_cast<size_t>(p.stage_cap));
     st = ensure_smem_attr(dev, 9, dsa::topk_kernel<512>, static_cast<int>(kMaxSmemPerBlock));
     if (st != DSA_OK) return st;
-    dsa::topk_kernel<512><<<d->T, 512, smem, stream>>>(p);
+    if (launch_pdl(dsa::topk_kernel<512>, d->T, 512, smem, stream, 0, p) != cudaSuccess)
+      return DSA_ERR_CUDA;
   }
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }

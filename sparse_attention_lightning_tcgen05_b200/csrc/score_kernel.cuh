@@ -224,53 +224,14 @@ struct CtaRange {
   int64_t a_seqoff, f_seqoff;
 };
 
-// Inclusive warp scan of 64-bit counts.
-__device__ __forceinline__ int64_t warp_incl_scan64(int64_t v) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int64_t n = __shfl_up_sync(0xffffffffu, v, off);
-    if (lane >= off) v += n;
-  }
-  return v;
-}
-
-// POSITIONS: the block holding item `idx` of the active (fill == false) or
-// fill list, by a warp-wide scan over blocks. Executed by a full warp.
-__device__ __forceinline__ void locate_positions(const ScoreParams &p, int tqt, int64_t idx, bool fill,
-                                 int &b_out, int &j_out) {
-  const int lane = threadIdx.x & 31;
-  const int nqb = pos_num_blocks(p, tqt);
-  int64_t base = 0;
-  b_out = nqb;
-  j_out = 0;
-  for (int c0 = 0; c0 < nqb; c0 += 32) {
-    const int b = c0 + lane;
-    int64_t cnt = 0;
-    int act = 0;
-    if (b < nqb) {
-      QBlk q;
-      make_qb_positions(p, tqt, b, q);
-      act = q.act;
-      cnt = fill ? q.ntr - q.act : q.act;
-    }
-    const int64_t incl = warp_incl_scan64(cnt);
-    const int64_t total = __shfl_sync(0xffffffffu, incl, 31);
-    const unsigned hit = __ballot_sync(0xffffffffu, base + incl > idx);
-    if (hit) {
-      const int f = __ffs(hit) - 1;
-      const int64_t excl = __shfl_sync(0xffffffffu, incl - cnt, f);
-      const int act_f = __shfl_sync(0xffffffffu, act, f);
-      b_out = c0 + f;
-      j_out = static_cast<int>(idx - base - excl) + (fill ? act_f : 0);
-      return;
-    }
-    base += total;
-  }
-}
-
-// POSITIONS: total active and fill items (full warp).
-__device__ __forceinline__ void count_positions(const ScoreParams &p, int tqt, int64_t &A, int64_t &F) {
+// POSITIONS: this CTA's share of both lists in two warp-wide passes over the
+// query blocks. Pass 1 sums the active and fill tiles; each lane 0..3 then
+// forms one bound (A*c/G, A*(c+1)/G, F*c/G, F*(c+1)/G) so that the four
+// divisions overlap. Pass 2 scans the blocks again, 32 at a time, and finds
+// the blocks holding items a0 and f0. A chunk of 32 blocks holds fewer than
+// 2^29 tiles (a row has at most 2^24), so the scans inside a chunk are
+// 32-bit; only the running bases are 64-bit. Full warp.
+__device__ __forceinline__ void cta_range_positions(const ScoreParams &p, int tqt, CtaRange &R) {
   const int lane = threadIdx.x & 31;
   const int nqb = pos_num_blocks(p, tqt);
   int64_t a = 0, f = 0;
@@ -285,8 +246,57 @@ __device__ __forceinline__ void count_positions(const ScoreParams &p, int tqt, i
     a += __shfl_xor_sync(0xffffffffu, a, off);
     f += __shfl_xor_sync(0xffffffffu, f, off);
   }
-  A = a;
-  F = f;
+  int64_t bound = 0;
+  if (lane < 4) bound = (lane < 2 ? a : f) * (blockIdx.x + (lane & 1)) / gridDim.x;
+  const int64_t a0 = __shfl_sync(0xffffffffu, bound, 0);
+  const int64_t a1 = __shfl_sync(0xffffffffu, bound, 1);
+  const int64_t f0 = __shfl_sync(0xffffffffu, bound, 2);
+  const int64_t f1 = __shfl_sync(0xffffffffu, bound, 3);
+  R.a_count = a1 - a0;
+  R.f_count = f1 - f0;
+  R.a_seq = R.f_seq = 0;
+  R.a_b = R.f_b = nqb;
+  R.a_j = R.f_j = 0;
+  R.a_seqoff = R.f_seqoff = 0;
+  bool need_a = R.a_count > 0, need_f = R.f_count > 0;
+  int64_t abase = 0, fbase = 0;
+  for (int c0 = 0; c0 < nqb && (need_a || need_f); c0 += 32) {
+    const int b = c0 + lane;
+    int act = 0, fil = 0;
+    if (b < nqb) {
+      QBlk q;
+      make_qb_positions(p, tqt, b, q);
+      act = q.act;
+      fil = q.ntr - q.act;
+    }
+    int ia = act, jf = fil;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int na = __shfl_up_sync(0xffffffffu, ia, off);
+      const int nf = __shfl_up_sync(0xffffffffu, jf, off);
+      if (lane >= off) {
+        ia += na;
+        jf += nf;
+      }
+    }
+    const unsigned hit_a = __ballot_sync(0xffffffffu, need_a && abase + ia > a0);
+    const unsigned hit_f = __ballot_sync(0xffffffffu, need_f && fbase + jf > f0);
+    if (hit_a) {
+      const int l = __ffs(hit_a) - 1;
+      R.a_b = c0 + l;
+      R.a_j = static_cast<int>(a0 - abase - __shfl_sync(0xffffffffu, ia - act, l));
+      need_a = false;
+    }
+    if (hit_f) {
+      const int l = __ffs(hit_f) - 1;
+      R.f_b = c0 + l;
+      R.f_j = static_cast<int>(f0 - fbase - __shfl_sync(0xffffffffu, jf - fil, l)) +
+              __shfl_sync(0xffffffffu, act, l);
+      need_f = false;
+    }
+    abase += __shfl_sync(0xffffffffu, ia, 31);
+    fbase += __shfl_sync(0xffffffffu, jf, 31);
+  }
 }
 
 // CAUSAL: active or fill items before block B of a sequence.
@@ -342,10 +352,13 @@ __device__ __forceinline__ void count_causal(const ScoreParams &p, int tqt, int6
 // This CTA's share of both lists (executed by a full warp; every lane gets
 // the same result).
 __device__ __forceinline__ void cta_range(const ScoreParams &p, int tqt, CtaRange &R) {
+  if (p.mode == kModePositions) {
+    cta_range_positions(p, tqt, R);
+    return;
+  }
   const int64_t G = gridDim.x, c = blockIdx.x;
   int64_t A = 0, F = 0;
-  if (p.mode == kModePositions) count_positions(p, tqt, A, F);
-  else count_causal(p, tqt, A, F);
+  count_causal(p, tqt, A, F);
   const int64_t a0 = A * c / G, a1 = A * (c + 1) / G;
   const int64_t f0 = F * c / G, f1 = F * (c + 1) / G;
   R.a_count = a1 - a0;
@@ -354,13 +367,8 @@ __device__ __forceinline__ void cta_range(const ScoreParams &p, int tqt, CtaRang
   R.a_b = R.f_b = 0;
   R.a_j = R.f_j = 0;
   R.a_seqoff = R.f_seqoff = 0;
-  if (p.mode == kModePositions) {
-    if (R.a_count > 0) locate_positions(p, tqt, a0, false, R.a_b, R.a_j);
-    if (R.f_count > 0) locate_positions(p, tqt, f0, true, R.f_b, R.f_j);
-  } else {
-    if (R.a_count > 0) locate_causal(p, tqt, a0, false, R.a_seq, R.a_b, R.a_j, R.a_seqoff);
-    if (R.f_count > 0) locate_causal(p, tqt, f0, true, R.f_seq, R.f_b, R.f_j, R.f_seqoff);
-  }
+  if (R.a_count > 0) locate_causal(p, tqt, a0, false, R.a_seq, R.a_b, R.a_j, R.a_seqoff);
+  if (R.f_count > 0) locate_causal(p, tqt, f0, true, R.f_seq, R.f_b, R.f_j, R.f_seqoff);
 }
 
 __device__ __forceinline__ void make_qb(const ScoreParams &p, int tqt, int seq, int b,
@@ -498,6 +506,27 @@ __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
                          tmem_cols_needed(kNACC, n_cols, kSTAGES, kQBUF, kNSUB, kFP8)))
     tmem_cols <<= 1;
 
+  // Set-up that reads nothing written by earlier work on the stream runs
+  // before the dependency wait, overlapping the previous kernel's tail.
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < kSTAGES; ++i) { mbar_init(full_k + i, 1); mbar_init(empty_k + i, 1); }
+    for (int i = 0; i < kQBUF; ++i) { mbar_init(q_full + i, 1); mbar_init(q_empty + i, 1); }
+    for (int i = 0; i < kNACC; ++i) { mbar_init(acc_full + i, 1); mbar_init(acc_empty + i, kEPI); }
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmap_k);
+    tma_prefetch_desc(&tmap_q);
+    if constexpr (kFP8) {
+      tma_prefetch_desc(&tmap_ksf);
+      tma_prefetch_desc(&tmap_qsf);
+    }
+  } else if (warp == 1) {
+    tmem_alloc(tmem_base_slot, tmem_cols);
+    tmem_relinquish();
+  }
+  grid_dep_wait();
+  grid_dep_launch_dependents();
+
   // Decode positions are read by every role many times: keep a copy here.
   int *spos = reinterpret_cast<int *>(smem + L.off_pos);
   const bool pos_staged = p.mode == kModePositions && p.T <= kPosCap;
@@ -506,27 +535,10 @@ __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
   __syncthreads();
   ScoreParams P = p;
   if (pos_staged) P.positions = spos;
-
   if (warp == 0) {
     CtaRange R;
     cta_range(P, tqt, R);
-    if (lane == 0) {
-      *range_slot = R;
-      for (int i = 0; i < kSTAGES; ++i) { mbar_init(full_k + i, 1); mbar_init(empty_k + i, 1); }
-      for (int i = 0; i < kQBUF; ++i) { mbar_init(q_full + i, 1); mbar_init(q_empty + i, 1); }
-      for (int i = 0; i < kNACC; ++i) { mbar_init(acc_full + i, 1); mbar_init(acc_empty + i, kEPI); }
-      *abort_flag = 0;
-      fence_mbar_init();
-      tma_prefetch_desc(&tmap_k);
-      tma_prefetch_desc(&tmap_q);
-      if constexpr (kFP8) {
-        tma_prefetch_desc(&tmap_ksf);
-        tma_prefetch_desc(&tmap_qsf);
-      }
-    }
-  } else if (warp == 1) {
-    tmem_alloc(tmem_base_slot, tmem_cols);
-    tmem_relinquish();
+    if (lane == 0) *range_slot = R;
   }
   tc_fence_before_sync();
   __syncthreads();

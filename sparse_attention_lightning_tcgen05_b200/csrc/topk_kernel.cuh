@@ -23,6 +23,8 @@
 
 #include <cstdint>
 
+#include "sm100_ptx.cuh"
+
 namespace dsa {
 
 constexpr int kTopkBins = 2048;          // first-digit bins (11 bits)
@@ -68,9 +70,8 @@ __device__ __forceinline__ uint32_t score_key(float f) {
 }
 
 // Inclusive block-wide prefix sum of v; *total receives the block sum.
-template <int NT>
-__device__ __forceinline__ uint32_t block_incl_scan(uint32_t v, TopkShared<NT> &sm,
-                                                    uint32_t *total) {
+template <int NT, typename SM>
+__device__ __forceinline__ uint32_t block_incl_scan(uint32_t v, SM &sm, uint32_t *total) {
   constexpr int kWarps = NT / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
@@ -97,8 +98,8 @@ __device__ __forceinline__ uint32_t block_incl_scan(uint32_t v, TopkShared<NT> &
 }
 
 // Block-wide min and max of the keys each thread saw (into sm.kmin/kmax).
-template <int NT>
-__device__ __forceinline__ void block_minmax(uint32_t lo, uint32_t hi, TopkShared<NT> &sm) {
+template <int NT, typename SM>
+__device__ __forceinline__ void block_minmax(uint32_t lo, uint32_t hi, SM &sm) {
   constexpr int kWarps = NT / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
@@ -129,22 +130,23 @@ __device__ __forceinline__ void block_minmax(uint32_t lo, uint32_t hi, TopkShare
 
 // The bin b holding the need-th largest entry: sum(hist[b+1..]) < need <=
 // sum(hist[b..]). Writes sm.sel_bin and sm.sel_above = sum(hist[b+1..]).
-template <int NT>
-__device__ __forceinline__ void select_bin(TopkShared<NT> &sm, uint32_t need, int nbins) {
+template <int NT, typename SM>
+__device__ __forceinline__ void select_bin(SM &sm, const uint32_t *hist, uint32_t need,
+                                           int nbins) {
   constexpr int kPer = (kTopkBins + NT - 1) / NT;
   const int b0 = threadIdx.x * kPer;
   uint32_t own = 0;
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) own += (b0 + i < nbins) ? sm.hist[b0 + i] : 0u;
+  for (int i = 0; i < kPer; ++i) own += (b0 + i < nbins) ? hist[b0 + i] : 0u;
   uint32_t total;
-  const uint32_t incl = block_incl_scan(own, sm, &total);
+  const uint32_t incl = block_incl_scan<NT>(own, sm, &total);
   const uint32_t suffix_from_me = total - (incl - own);   // bins >= b0
   const uint32_t suffix_after_me = suffix_from_me - own;  // bins >= b0 + kPer
   if (own > 0 && suffix_after_me < need && need <= suffix_from_me) {
     uint32_t acc = suffix_after_me;
 #pragma unroll
     for (int i = kPer - 1; i >= 0; --i) {
-      const uint32_t h = (b0 + i < nbins) ? sm.hist[b0 + i] : 0u;
+      const uint32_t h = (b0 + i < nbins) ? hist[b0 + i] : 0u;
       if (acc + h >= need) {
         sm.sel_bin = b0 + i;
         sm.sel_above = acc;
@@ -214,7 +216,7 @@ __device__ void stage_row(const float *row, uint32_t n, float *keys, TopkShared<
     lo = min(lo, kk);
     hi = max(hi, kk);
   }
-  block_minmax(lo, hi, sm);
+  block_minmax<NT>(lo, hi, sm);
 }
 
 template <int NT>
@@ -224,6 +226,9 @@ __global__ void __launch_bounds__(NT) topk_kernel(const TopkParams p) {
   float *staged_keys = reinterpret_cast<float *>(smem_raw + sizeof(TopkShared<NT>));
   const int t = blockIdx.x;
   const int tid = threadIdx.x;
+  // scores (and positions) come from earlier work on the stream
+  grid_dep_wait();
+  grid_dep_launch_dependents();
 
   // ---- row geometry ----
   const float *row;
@@ -297,7 +302,7 @@ __global__ void __launch_bounds__(NT) topk_kernel(const TopkParams p) {
       atomicAdd(&sm.hist[value_bin(src.val(s), vmin, vscale)], 1u);
     }
     __syncthreads();
-    select_bin(sm, need, kTopkBins);
+    select_bin<NT>(sm, sm.hist, need, kTopkBins);
     const int b1 = static_cast<int>(sm.sel_bin);
     need -= sm.sel_above;
     n_match = sm.hist[b1];
@@ -353,7 +358,7 @@ __global__ void __launch_bounds__(NT) topk_kernel(const TopkParams p) {
       }
     }
     __syncthreads();
-    select_bin(sm, need, 1 << dbits);
+    select_bin<NT>(sm, sm.hist, need, 1 << dbits);
     const uint32_t b = sm.sel_bin;
     need -= sm.sel_above;
     prefix = (lo_bit >= 32 ? 0u : (prefix << dbits)) | b;
@@ -482,7 +487,7 @@ __global__ void __launch_bounds__(NT) topk_kernel(const TopkParams p) {
     }
     const uint32_t own = (__popc(gt) << 16) | __popc(eq);
     uint32_t total;
-    const uint32_t excl = block_incl_scan(own, sm, &total) - own;
+    const uint32_t excl = block_incl_scan<NT>(own, sm, &total) - own;
     const uint32_t E0 = base_eq + (excl & 0xFFFFu);
     uint32_t E = E0;
     uint32_t pos = base_gt + (excl >> 16) + min(E0, need);

@@ -138,16 +138,18 @@ dsa_status_t make_map(CUtensorMap *m, CUtensorMapDataType dt, cuuint32_t rank, c
   return r == CUDA_SUCCESS ? DSA_OK : DSA_ERR_INVALID_ARG;
 }
 
-// One kernel choice: template instance, its sub-block geometry.
+// One kernel choice: template instance and its geometry.
 using ScoreKernelFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
                                const CUtensorMap, const ScoreParams);
 struct ScoreLaunch {
   ScoreKernelFn kernel;
   uint32_t attr_bit;
-  int stages, qbuf, nsub, threads;
+  int stages, qbuf, nsub, epi, tiles, issuers;   // as the template arguments
   int tq_sub, n_cols;
   int max_cols;   // widest query block this instance ever runs (smem attribute)
   bool fp8;
+  // producer, MMA, epilogue warps, (fp8) scale warp, second issuer
+  int threads() const { return (2 + epi + (fp8 ? 1 : 0) + (issuers - 1)) * 32; }
 };
 
 // Launch with programmatic stream serialisation: the kernel may start while
@@ -186,31 +188,34 @@ int pow2_floor(int x) {
   return p;
 }
 
+// Kernel instances. Decode with one cache per token (H = 64): two key tiles
+// per pipeline item. Prefill / a shared cache (H = 64): 8 tokens per query
+// block as two N = 256 sub-blocks. Any other H: the generic epilogue.
 ScoreLaunch choose_score(const dsa_indexer_desc_t *d) {
   const bool per_token_cache = d->mask == DSA_MASK_POSITIONS && d->k_seq_stride != 0;
   const int H = d->H;
   if (d->dtype == DSA_KV_BF16) {
     if (per_token_cache) {
       if (H == 64)
-        return {dsa::score_kernel<64, 1, 4, 5, 2, 4, false>, 0, 5, 2, 1, 6 * 32, 1, 64, 64, false};
-      return {dsa::score_kernel<0, 1, 2, 4, 1, 4, false>, 1, 4, 1, 1, 6 * 32, 1, round16(H), 256,
+        return {dsa::score_kernel<64, 1, 2, 3, 2, 2, 8, false, 2>, 0, 2, 2, 1, 8, 2, 2, 1, 64, 64, false};
+      return {dsa::score_kernel<0, 1, 1, 2, 4, 1, 4, false, 1>, 1, 4, 1, 1, 4, 1, 1, 1, round16(H), 256,
               false};
     }
     if (H == 64)
-      return {dsa::score_kernel<64, 2, 2, 2, 1, 8, false>, 2, 2, 1, 2, 10 * 32, 4, 256, 256, false};
+      return {dsa::score_kernel<64, 2, 1, 2, 2, 1, 8, false, 1>, 2, 2, 1, 2, 8, 1, 1, 4, 256, 256, false};
     const int tq = pow2_floor(std::min(128, 256 / H));
-    return {dsa::score_kernel<0, 1, 2, 4, 1, 4, false>, 1, 4, 1, 1, 6 * 32, tq, round16(tq * H), 256,
-            false};
+    return {dsa::score_kernel<0, 1, 1, 2, 4, 1, 4, false, 1>, 1, 4, 1, 1, 4, 1, 1, tq, round16(tq * H),
+            256, false};
   }
   if (per_token_cache) {
     if (H == 64)
-      return {dsa::score_kernel<64, 1, 4, 8, 2, 4, true>, 3, 8, 2, 1, 6 * 32, 1, 64, 64, true};
-    return {dsa::score_kernel<0, 1, 2, 4, 1, 4, true>, 4, 4, 1, 1, 6 * 32, 1, round16(H), 128, true};
+      return {dsa::score_kernel<64, 1, 2, 3, 5, 2, 8, true, 2>, 3, 5, 2, 1, 8, 2, 2, 1, 64, 64, true};
+    return {dsa::score_kernel<0, 1, 1, 2, 4, 1, 4, true, 1>, 4, 4, 1, 1, 4, 1, 1, 1, round16(H), 128, true};
   }
   if (H == 64)
-    return {dsa::score_kernel<64, 2, 2, 4, 1, 8, true>, 5, 4, 1, 2, 10 * 32, 2, 128, 128, true};
+    return {dsa::score_kernel<64, 2, 1, 2, 4, 1, 8, true, 1>, 5, 4, 1, 2, 8, 1, 1, 2, 128, 128, true};
   const int tq = pow2_floor(std::min(128, 128 / H));
-  return {dsa::score_kernel<0, 1, 2, 4, 1, 4, true>, 4, 4, 1, 1, 6 * 32, tq, round16(tq * H), 128,
+  return {dsa::score_kernel<0, 1, 1, 2, 4, 1, 4, true, 1>, 4, 4, 1, 1, 4, 1, 1, tq, round16(tq * H), 128,
           true};
 }
 
@@ -222,9 +227,9 @@ dsa_status_t launch_score(const dsa_indexer_desc_t *d, const void *q, const uint
   dsa_status_t st = device_info(&dev);
   if (st != DSA_OK) return st;
   const ScoreLaunch L = choose_score(d);
-  const ScoreSmem plan(L.stages, L.qbuf, L.nsub, L.n_cols, L.fp8);
+  const ScoreSmem plan(L.stages, L.qbuf, L.nsub, L.n_cols, L.fp8, L.epi, L.tiles);
   // the attribute is set once per kernel: use the widest query block it runs
-  const ScoreSmem widest(L.stages, L.qbuf, L.nsub, L.max_cols, L.fp8);
+  const ScoreSmem widest(L.stages, L.qbuf, L.nsub, L.max_cols, L.fp8, L.epi, L.tiles);
   if (widest.total > kMaxSmemPerBlock || plan.total > widest.total) return DSA_ERR_UNSUPPORTED;
   st = ensure_smem_attr(dev, L.attr_bit, L.kernel, static_cast<int>(widest.total));
   if (st != DSA_OK) return st;
@@ -298,7 +303,7 @@ dsa_status_t launch_score(const dsa_indexer_desc_t *d, const void *q, const uint
     const int64_t nqb = p.shared_cache ? (d->T + tqt - 1) / tqt : d->T;
     if (nqb * ntiles < grid) grid = static_cast<int>(nqb * ntiles);
   }
-  if (launch_pdl(L.kernel, grid, L.threads, plan.total, stream, 0, tk, tq, tksf, tqsf, p) !=
+  if (launch_pdl(L.kernel, grid, L.threads(), plan.total, stream, 0, tk, tq, tksf, tqsf, p) !=
       cudaSuccess)
     return DSA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;

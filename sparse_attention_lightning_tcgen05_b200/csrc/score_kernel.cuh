@@ -86,12 +86,15 @@ __host__ __device__ constexpr uint32_t sf_raw_bytes_q(int n_cols) {
 constexpr int kPosCap = 2048;          // positions staged in shared memory
 constexpr int kWRowsPerWarp = 4;        // H=64 epilogue: w rows a warp keeps
 
+// A stage holds `tiles` key tiles (one pipeline item); each tile slot has
+// its own data and (fp8) scale window.
 struct ScoreSmem {
   uint32_t k_stage_bytes, k_sf_bytes, q_sub_bytes, q_sf_bytes;
   uint32_t off_k, off_ksf, off_q, off_qsf, off_w, off_pos, off_bar, off_misc, total;
   __host__ __device__ ScoreSmem(int stages, int qbuf, int nsub, int n_cols, bool fp8,
-                                int epi_warps = 8) {
+                                int epi_warps, int tiles) {
     // bf16: two 128-byte-wide halves along D; fp8: one 128-byte row.
+    // (k_stage_bytes / k_sf_bytes are per tile slot.)
     k_stage_bytes = fp8 ? kBlockM * 128 : kBlockM * 256;
     q_sub_bytes = fp8 ? n_cols * 128 : n_cols * 256;
     // fp8 scale words (4 bytes a row) as loaded -- a window of rows + 4 words
@@ -100,9 +103,9 @@ struct ScoreSmem {
     k_sf_bytes = fp8 ? kSfRawBytesK + 512 : 0;
     q_sf_bytes = fp8 ? static_cast<uint32_t>(sf_raw_bytes_q(n_cols) + sf_atoms(n_cols) * 512) : 0;
     off_k = 0;
-    off_q = off_k + stages * k_stage_bytes;
+    off_q = off_k + stages * tiles * k_stage_bytes;
     off_ksf = off_q + qbuf * nsub * q_sub_bytes;
-    off_qsf = off_ksf + stages * k_sf_bytes;
+    off_qsf = off_ksf + stages * tiles * k_sf_bytes;
     off_w = off_qsf + qbuf * nsub * q_sf_bytes;
     off_w = (off_w + 15) & ~15u;
     off_pos = off_w + epi_warps * kWRowsPerWarp * 64 * 4;
@@ -112,11 +115,14 @@ struct ScoreSmem {
   }
 };
 
-// TMEM columns: accumulators, then (fp8) per-stage A scales, then per
-// query-buffer sub-block B scales.
-__host__ __device__ constexpr int tmem_cols_needed(int nacc, int n_cols, int stages,
-                                                  int qbuf, int nsub, bool fp8) {
-  return nacc * n_cols + (fp8 ? stages * 4 + qbuf * nsub * 4 * sf_atoms(n_cols) : 0);
+// TMEM columns: accumulator slots (acc_per_slot accumulators of n_cols each),
+// then (fp8) A scales per stage tile slot, then B scales per query-buffer
+// sub-block.
+__host__ __device__ constexpr int tmem_cols_needed(int nacc, int acc_per_slot, int n_cols,
+                                                  int stages, int tiles, int qbuf, int nsub,
+                                                  bool fp8) {
+  return nacc * acc_per_slot * n_cols +
+         (fp8 ? stages * tiles * 4 + qbuf * nsub * 4 * sf_atoms(n_cols) : 0);
 }
 
 // ---- the static schedule --------------------------------------------------------
@@ -377,25 +383,48 @@ __device__ __forceinline__ void make_qb(const ScoreParams &p, int tqt, int seq, 
   else make_qb_causal(p, tqt, seq, b, seqoff, q);
 }
 
-// Advance an active cursor by one item: the next tile, or the first tile of
-// the next block that has one. False past the end of the list.
-__device__ __forceinline__ bool next_active(const ScoreParams &p, int tqt, QBlk &q, int &j) {
-  if (++j < q.act) return true;
+// A walk over this CTA's share of the active list, one pipeline item at a
+// time: up to kG consecutive key tiles of one query block. Every role walks
+// the same items in the same order.
+struct ItemCursor {
+  QBlk q;
+  int j;          // first tile of the current item
+  int64_t left;   // tiles of the share not yet taken
+};
+
+__device__ __forceinline__ void cursor_start(const ScoreParams &p, int tqt, const CtaRange &R,
+                                             ItemCursor &c) {
+  make_qb(p, tqt, R.a_seq, R.a_b, R.a_seqoff, c.q);
+  c.j = R.a_j;
+  c.left = R.a_count;
+}
+
+// Tiles of the current item.
+template <int kG>
+__device__ __forceinline__ int cursor_tiles(const ItemCursor &c) {
+  const int in_block = c.q.act - c.j < kG ? c.q.act - c.j : kG;
+  return c.left < in_block ? static_cast<int>(c.left) : in_block;
+}
+
+// Step past the g tiles of the current item. True when the walk left the
+// query block (or the share is used up).
+__device__ __forceinline__ bool cursor_next_block(const ScoreParams &p, int tqt, ItemCursor &c) {
   do {
-    if (!next_qb(p, tqt, q)) return false;
-  } while (q.act == 0);
-  j = 0;
+    if (!next_qb(p, tqt, c.q)) {
+      c.left = 0;
+      return true;
+    }
+  } while (c.q.act == 0);
+  c.j = 0;
   return true;
 }
 
-// Advance a fill cursor by one item.
-__device__ __forceinline__ bool next_fill(const ScoreParams &p, int tqt, QBlk &q, int &j) {
-  if (++j < q.ntr) return true;
-  do {
-    if (!next_qb(p, tqt, q)) return false;
-  } while (q.act == q.ntr);
-  j = q.act;
-  return true;
+__device__ __forceinline__ bool cursor_step(const ScoreParams &p, int tqt, ItemCursor &c, int g) {
+  c.j += g;
+  c.left -= g;
+  if (c.left <= 0) return true;
+  if (c.j < c.q.act) return false;
+  return cursor_next_block(p, tqt, c);
 }
 
 // ---- epilogue helpers ---------------------------------------------------------------
@@ -462,11 +491,20 @@ __device__ __forceinline__ void sf_reorder_atom(const uint32_t *rows, int nrows,
 
 // kH: 64 selects the tuned epilogue; 0 = any H (generic epilogue).
 // kNSUB: MMA sub-blocks per key tile (each its own accumulator, same A).
-// kNACC: TMEM accumulator buffers. kSTAGES: key-tile smem stages.
+// kG: key tiles per pipeline item (one smem stage, one accumulator slot of
+//     kG accumulators); kG > 1 needs kNSUB == 1. Batching tiles amortises
+//     the per-item waits, fences and commits of the issuing threads.
+// kNACC: TMEM accumulator slots. kSTAGES: smem stages (kG tiles each).
 // kQBUF: query-block smem buffers. kEPI: epilogue warps (4 or 8).
 // kFP8: e4m3 + e8m0/32 inputs through the block-scaled MMA.
-template <int kH, int kNSUB, int kNACC, int kSTAGES, int kQBUF, int kEPI, bool kFP8>
-__global__ void __launch_bounds__((2 + kEPI) * 32, 1)
+// kISS: MMA-issuing warps (1 or 2). With 2, items alternate between them so
+//     that one warp's waits and commits overlap the other's MMAs.
+//
+// Warps: 0 TMA producer, 1 MMA issuer (+ TMEM owner), 2 .. 1+kEPI epilogue,
+// then (fp8) the scale-factor warp, then (kISS == 2) the second issuer.
+template <int kH, int kNSUB, int kG, int kNACC, int kSTAGES, int kQBUF, int kEPI, bool kFP8,
+          int kISS>
+__global__ void __launch_bounds__((2 + kEPI + (kFP8 ? 1 : 0) + (kISS - 1)) * 32, 1)
     score_kernel(const __grid_constant__ CUtensorMap tmap_k,
                  const __grid_constant__ CUtensorMap tmap_q,
                  const __grid_constant__ CUtensorMap tmap_ksf,
@@ -474,12 +512,17 @@ __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
                  const ScoreParams p) {
   static_assert(kEPI == 4 || kEPI == 8, "epilogue warps");
   static_assert(kH == 64 || kEPI == 4, "generic epilogue uses 4 warps");
-  static_assert(2 * (kSTAGES + kQBUF + kNACC) <= 64, "barrier budget");
+  static_assert(kG == 1 || kNSUB == 1, "tile batching is for single sub-block queries");
+  static_assert(kISS == 1 || kISS == 2, "issuers");
+  constexpr int kSFWarp = 2 + kEPI;                        // fp8 scale-factor warp
+  constexpr int kIss2Warp = 2 + kEPI + (kFP8 ? 1 : 0);     // second MMA issuer
+  static_assert(3 * (kSTAGES + kQBUF) + 2 * kNACC <= 64, "barrier budget");
   constexpr int kGroups = kEPI / 4;
+  constexpr int kAPS = kG;                       // accumulators per slot
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const ScoreSmem L(kSTAGES, kQBUF, kNSUB, p.n_cols, kFP8, kEPI);
+  const ScoreSmem L(kSTAGES, kQBUF, kNSUB, p.n_cols, kFP8, kEPI, kG);
   uint8_t *sk = smem + L.off_k;
   uint8_t *sq = smem + L.off_q;
   uint8_t *sksf = smem + L.off_ksf;
@@ -491,6 +534,8 @@ __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
   uint64_t *q_empty = q_full + kQBUF;            // [kQBUF]
   uint64_t *acc_full = q_empty + kQBUF;          // [kNACC]
   uint64_t *acc_empty = acc_full + kNACC;        // [kNACC]
+  uint64_t *sf_ready = acc_empty + kNACC;        // [kSTAGES] fp8: A scales in TMEM
+  uint64_t *sfq_ready = sf_ready + kSTAGES;      // [kQBUF]   fp8: B scales in TMEM
   uint32_t *misc = reinterpret_cast<uint32_t *>(smem + L.off_misc);
   uint32_t *tmem_base_slot = misc;               // written by tcgen05.alloc
   volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 1);
@@ -502,16 +547,20 @@ __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
   const int n_cols = p.n_cols;
   const int atoms = sf_atoms(n_cols);
   uint32_t tmem_cols = 32;
-  while (tmem_cols < static_cast<uint32_t>(
-                         tmem_cols_needed(kNACC, n_cols, kSTAGES, kQBUF, kNSUB, kFP8)))
+  while (tmem_cols < static_cast<uint32_t>(tmem_cols_needed(kNACC, kAPS, n_cols, kSTAGES, kG,
+                                                            kQBUF, kNSUB, kFP8)))
     tmem_cols <<= 1;
 
   // Set-up that reads nothing written by earlier work on the stream runs
   // before the dependency wait, overlapping the previous kernel's tail.
   if (warp == 0 && lane == 0) {
     for (int i = 0; i < kSTAGES; ++i) { mbar_init(full_k + i, 1); mbar_init(empty_k + i, 1); }
-    for (int i = 0; i < kQBUF; ++i) { mbar_init(q_full + i, 1); mbar_init(q_empty + i, 1); }
+    for (int i = 0; i < kQBUF; ++i) { mbar_init(q_full + i, 1); mbar_init(q_empty + i, kISS); }
     for (int i = 0; i < kNACC; ++i) { mbar_init(acc_full + i, 1); mbar_init(acc_empty + i, kEPI); }
+    if constexpr (kFP8) {
+      for (int i = 0; i < kSTAGES; ++i) mbar_init(sf_ready + i, 1);
+      for (int i = 0; i < kQBUF; ++i) mbar_init(sfq_ready + i, 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmap_k);
@@ -546,27 +595,28 @@ __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
   const uint32_t tmem_base = *tmem_base_slot;
   const CtaRange R = *range_slot;
   const WaitCtl ctl{abort_flag, p.err, p.err_info, p.wait_limit_ns};
-  const uint32_t sfa_col0 = kNACC * n_cols;                    // fp8 only
-  const uint32_t sfb_col0 = sfa_col0 + kSTAGES * 4;            // fp8 only
+  const uint32_t sfa_col0 = kNACC * kAPS * n_cols;             // fp8 only
+  const uint32_t sfb_col0 = sfa_col0 + kSTAGES * kG * 4;       // fp8 only
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0 && R.a_count > 0) {
       Ring st, qb;
       uint32_t k_issued = 0, q_issued = 0, k_last_phase = 0, q_last_phase = 0;
-      QBlk q;
-      int j = R.a_j;
-      make_qb(P, tqt, R.a_seq, R.a_b, R.a_seqoff, q);
+      ItemCursor c;
+      cursor_start(P, tqt, R, c);
+      const uint32_t tile_tx = L.k_stage_bytes + (kFP8 ? kSfBoxBytesK : 0);
       bool need_q = true;
-      for (int64_t n = 0; n < R.a_count; ++n) {
+      while (c.left > 0) {
+        const int g = cursor_tiles<kG>(c);
         if (need_q) {
-          const int nsub = (q.ntok + p.tq_sub - 1) / p.tq_sub;
+          const int nsub = (c.q.ntok + p.tq_sub - 1) / p.tq_sub;
           if (!mbar_wait(q_empty + qb.idx, qb.phase ^ 1u, ctl, 2)) break;
           mbar_arrive_expect_tx(q_full + qb.idx,
                                 nsub * (L.q_sub_bytes + (kFP8 ? sf_box_bytes_q(n_cols) : 0)));
           for (int s = 0; s < nsub; ++s) {
             uint8_t *dst = sq + (qb.idx * kNSUB + s) * L.q_sub_bytes;
-            const int row = (q.t0 + s * p.tq_sub) * p.H;
+            const int row = (c.q.t0 + s * p.tq_sub) * p.H;
             if constexpr (kFP8) {
               tma_load_2d(dst, &tmap_q, q_full + qb.idx, 0, row);
               tma_load_2d(sqsf + (qb.idx * kNSUB + s) * L.q_sf_bytes, &tmap_qsf,
@@ -581,24 +631,24 @@ __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
           need_q = false;
         }
         if (!mbar_wait(empty_k + st.idx, st.phase ^ 1u, ctl, 3)) break;
-        mbar_arrive_expect_tx(full_k + st.idx, L.k_stage_bytes + (kFP8 ? kSfBoxBytesK : 0));
-        uint8_t *dst = sk + st.idx * L.k_stage_bytes;
-        const int y = q.y0 + j * kBlockM;
-        if constexpr (kFP8) {
-          tma_load_3d(dst, &tmap_k, full_k + st.idx, 0, y, q.z);
-          tma_load_2d(sksf + st.idx * L.k_sf_bytes, &tmap_ksf, full_k + st.idx,
-                      y & ~(kSfPad - 1), q.z);
-        } else {
-          tma_load_3d(dst, &tmap_k, full_k + st.idx, 0, y, q.z);
-          tma_load_3d(dst + kBlockM * 128, &tmap_k, full_k + st.idx, 64, y, q.z);
+        mbar_arrive_expect_tx(full_k + st.idx, g * tile_tx);
+        for (int i = 0; i < g; ++i) {
+          uint8_t *dst = sk + (st.idx * kG + i) * L.k_stage_bytes;
+          const int y = c.q.y0 + (c.j + i) * kBlockM;
+          tma_load_3d(dst, &tmap_k, full_k + st.idx, 0, y, c.q.z);
+          if constexpr (kFP8) {
+            tma_load_2d(sksf + (st.idx * kG + i) * L.k_sf_bytes, &tmap_ksf, full_k + st.idx,
+                        y & ~(kSfPad - 1), c.q.z);
+          } else {
+            tma_load_3d(dst + kBlockM * 128, &tmap_k, full_k + st.idx, 64, y, c.q.z);
+          }
         }
         k_issued |= 1u << st.idx;
         k_last_phase = (k_last_phase & ~(1u << st.idx)) | (st.phase << st.idx);
         st.next(kSTAGES);
-        if (n + 1 < R.a_count) {
-          const int pb = q.b, ps = q.seq;
-          next_active(P, tqt, q, j);
-          if (q.b != pb || q.seq != ps) { need_q = true; qb.next(kQBUF); }
+        if (cursor_step(P, tqt, c, g) && c.left > 0) {
+          need_q = true;
+          qb.next(kQBUF);
         }
       }
       // Let every copy this thread started land before the CTA can exit.
@@ -607,87 +657,80 @@ __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
       for (int i = 0; i < kQBUF; ++i)
         if (q_issued >> i & 1u) mbar_drain(q_full + i, q_last_phase >> i & 1u, p.wait_limit_ns);
     }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer (whole warp walks the list) ----------------
+  } else if (warp == 1 || (kISS == 2 && warp == kIss2Warp)) {
+    // ---------------- MMA issuers (each walks every item, issues its own) ----
+    const int my_parity = warp == 1 ? 0 : 1;
     if (R.a_count > 0) {
       Ring st, qb, ac;
       uint64_t *last_commit = nullptr;
       uint32_t last_commit_phase = 0;
-      QBlk q;
-      int j = R.a_j;
-      make_qb(P, tqt, R.a_seq, R.a_b, R.a_seqoff, q);
+      ItemCursor c;
+      cursor_start(P, tqt, R, c);
       bool new_q = true;
-      for (int64_t n = 0; n < R.a_count; ++n) {
-        const int nsub = (q.ntok + p.tq_sub - 1) / p.tq_sub;
+      int nsub = 1;
+      // Shared-memory descriptors advance by (bytes >> 4) in their low field.
+      const uint64_t k_desc0 = sdesc_kmajor_sw128(smem_u32(sk));
+      const uint64_t q_desc0 = sdesc_kmajor_sw128(smem_u32(sq));
+      const uint32_t k_tile_step = L.k_stage_bytes >> 4;
+      const uint32_t q_sub_step = L.q_sub_bytes >> 4;
+      int item = 0;
+      while (c.left > 0) {
+        const int g = cursor_tiles<kG>(c);
+        const bool mine = kISS == 1 || (item & 1) == my_parity;
+        ++item;
         if (new_q) {
-          if (!mbar_wait(q_full + qb.idx, qb.phase, ctl, 12)) break;
-          if constexpr (kFP8) {
-            for (int s = 0; s < nsub; ++s) {
-              uint8_t *sf = sqsf + (qb.idx * kNSUB + s) * L.q_sf_bytes;
-              const int r = ((q.t0 + s * p.tq_sub) * p.H) & (kSfPad - 1);
-              for (int a = 0; a < atoms; ++a)
-                sf_reorder_atom(reinterpret_cast<const uint32_t *>(sf) + r + 128 * a,
-                                min(128, n_cols - 128 * a),
-                                reinterpret_cast<uint32_t *>(sf + sf_raw_bytes_q(n_cols) + 512 * a));
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              tc_fence_after_sync();
-              for (int s = 0; s < nsub; ++s) {
-                uint8_t *sf = sqsf + (qb.idx * kNSUB + s) * L.q_sf_bytes;
-                for (int a = 0; a < atoms; ++a)
-                  tmem_cp_32x128b_x4(
-                      tmem_base + sfb_col0 + (qb.idx * kNSUB + s) * 4 * atoms + 4 * a,
-                      sdesc_rows16_noswizzle(smem_u32(sf + sf_raw_bytes_q(n_cols) + 512 * a)));
-              }
-            }
-          }
+          nsub = (c.q.ntok + p.tq_sub - 1) / p.tq_sub;
+          // fp8: the scale warp has also put the block's B scales in TMEM
+          if (!mbar_wait(kFP8 ? sfq_ready + qb.idx : q_full + qb.idx, qb.phase, ctl, 12)) break;
           tc_fence_after_sync();
           new_q = false;
         }
-        if (!mbar_wait(full_k + st.idx, st.phase, ctl, 13)) break;
-        if constexpr (kFP8) {
-          uint8_t *sf = sksf + st.idx * L.k_sf_bytes;
-          const int r = (q.y0 + j * kBlockM) & (kSfPad - 1);
-          sf_reorder_atom(reinterpret_cast<const uint32_t *>(sf) + r, 128,
-                          reinterpret_cast<uint32_t *>(sf + kSfRawBytesK));
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tc_fence_after_sync();
-            tmem_cp_32x128b_x4(tmem_base + sfa_col0 + st.idx * 4,
-                               sdesc_rows16_noswizzle(smem_u32(sf + kSfRawBytesK)));
+        const int nslots = kG > 1 ? 1 : nsub;
+        if (!mine) {   // the other issuer's item: keep the rings in step
+          for (int s = 0; s < nslots; ++s) ac.next(kNACC);
+          st.next(kSTAGES);
+          if (cursor_step(P, tqt, c, g)) {
+            if (lane == 0) mma_commit(q_empty + qb.idx);
+            __syncwarp();
+            qb.next(kQBUF);
+            new_q = true;
           }
+          continue;
+        }
+        if (!mbar_wait(full_k + st.idx, st.phase, ctl, 13)) break;
+        if constexpr (kFP8) {   // and the item's A scales
+          if (!mbar_wait(sf_ready + st.idx, st.phase, ctl, 15)) break;
         }
         tc_fence_after_sync();
-        const uint32_t k_base = smem_u32(sk + st.idx * L.k_stage_bytes);
-        const uint32_t q_base = smem_u32(sq + qb.idx * kNSUB * L.q_sub_bytes);
         bool ok = true;
-        for (int s = 0; s < nsub; ++s) {
+        for (int s = 0; s < nslots; ++s) {
           if (!mbar_wait(acc_empty + ac.idx, ac.phase ^ 1u, ctl, 14)) { ok = false; break; }
           tc_fence_after_sync();
           if (lane == 0) {
-            const uint32_t d_tmem = tmem_base + ac.idx * n_cols;
-            const uint32_t qs = q_base + s * L.q_sub_bytes;
-            if constexpr (kFP8) {
-              const uint32_t sfa = tmem_base + sfa_col0 + st.idx * 4;
-              const uint32_t sfb = tmem_base + sfb_col0 + (qb.idx * kNSUB + s) * 4 * atoms;
+            const int sub = kG > 1 ? 0 : s;
+            const uint64_t bdesc = q_desc0 + (qb.idx * kNSUB + sub) * q_sub_step;
+            const int nacc = kG > 1 ? g : 1;
+            for (int i = 0; i < nacc; ++i) {
+              const uint32_t d_tmem = tmem_base + (ac.idx * kAPS + i) * n_cols;
+              const uint64_t adesc = k_desc0 + (st.idx * kG + i) * k_tile_step;
+              if constexpr (kFP8) {
+                const uint32_t sfa = tmem_base + sfa_col0 + (st.idx * kG + i) * 4;
+                const uint32_t sfb = tmem_base + sfb_col0 + (qb.idx * kNSUB + sub) * 4 * atoms;
+                const uint32_t idesc = idesc_mxf8_e4m3(kBlockM, n_cols, 0, 0);
 #pragma unroll
-              for (int kk = 0; kk < kHeadDim / 32; ++kk) {
-                const uint64_t ad = sdesc_kmajor_sw128(k_base + kk * 32);
-                const uint64_t bd = sdesc_kmajor_sw128(qs + kk * 32);
-                mma_mxf8_ss(d_tmem, ad, bd, idesc_mxf8_e4m3(kBlockM, n_cols, kk, kk), sfa, sfb,
-                            kk > 0 ? 1u : 0u);
-              }
-            } else {
-              const uint32_t idesc = idesc_bf16_f32(kBlockM, n_cols);
+                for (int kk = 0; kk < kHeadDim / 32; ++kk)
+                  mma_mxf8_ss(d_tmem, adesc + kk * 2, bdesc + kk * 2,
+                              idesc | idesc_mxf8_e4m3(0, 0, kk, kk), sfa, sfb, kk > 0 ? 1u : 0u);
+              } else {
+                const uint32_t idesc = idesc_bf16_f32(kBlockM, n_cols);
+                const uint32_t a_half = (kBlockM * 128) >> 4;
+                const uint32_t b_half = (n_cols * 128) >> 4;
 #pragma unroll
-              for (int kk = 0; kk < kHeadDim / 16; ++kk) {
-                const uint32_t half = kk / 4, koff = (kk % 4) * 32;
-                const uint64_t ad = sdesc_kmajor_sw128(k_base + half * (kBlockM * 128) + koff);
-                const uint64_t bd = sdesc_kmajor_sw128(qs + half * (n_cols * 128) + koff);
-                mma_f16_ss(d_tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
+                for (int kk = 0; kk < kHeadDim / 16; ++kk) {
+                  const uint32_t half = kk / 4, koff = (kk % 4) * 2;
+                  mma_f16_ss(d_tmem, adesc + half * a_half + koff, bdesc + half * b_half + koff,
+                             idesc, kk > 0 ? 1u : 0u);
+                }
               }
             }
             mma_commit(acc_full + ac.idx);
@@ -701,13 +744,7 @@ __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
         if (lane == 0) mma_commit(empty_k + st.idx);   // stage free once these MMAs finish
         __syncwarp();
         st.next(kSTAGES);
-        bool block_done = n + 1 == R.a_count;
-        if (!block_done) {
-          const int pb = q.b, ps = q.seq;
-          next_active(P, tqt, q, j);
-          block_done = q.b != pb || q.seq != ps;
-        }
-        if (block_done) {
+        if (cursor_step(P, tqt, c, g)) {
           if (lane == 0) mma_commit(q_empty + qb.idx);
           __syncwarp();
           qb.next(kQBUF);
@@ -718,7 +755,80 @@ __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
       if (lane == 0 && last_commit) mbar_drain(last_commit, last_commit_phase, p.wait_limit_ns);
       __syncwarp();
     }
-  } else {
+  } else if (kFP8 && warp == kSFWarp) {
+    // ---------------- fp8 scale factors ----------------
+    // Reorders each item's (and each query block's) scale words into the
+    // 128-row atoms tcgen05.cp copies, copies them into TMEM and commits to
+    // sf_ready / sfq_ready, so the MMA warp only waits and issues.
+    if (R.a_count > 0) {
+      Ring st, qb;
+      ItemCursor c;
+      cursor_start(P, tqt, R, c);
+      bool new_q = true;
+      uint64_t *last_commit = nullptr;
+      uint32_t last_commit_phase = 0;
+      while (c.left > 0) {
+        const int g = cursor_tiles<kG>(c);
+        if (new_q) {
+          const int nsub = (c.q.ntok + p.tq_sub - 1) / p.tq_sub;
+          if (!mbar_wait(q_full + qb.idx, qb.phase, ctl, 16)) break;
+          for (int s = 0; s < nsub; ++s) {
+            uint8_t *sf = sqsf + (qb.idx * kNSUB + s) * L.q_sf_bytes;
+            const int r = ((c.q.t0 + s * p.tq_sub) * p.H) & (kSfPad - 1);
+            for (int a = 0; a < atoms; ++a)
+              sf_reorder_atom(reinterpret_cast<const uint32_t *>(sf) + r + 128 * a,
+                              min(128, n_cols - 128 * a),
+                              reinterpret_cast<uint32_t *>(sf + sf_raw_bytes_q(n_cols) + 512 * a));
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tc_fence_after_sync();
+            for (int s = 0; s < nsub; ++s) {
+              uint8_t *sf = sqsf + (qb.idx * kNSUB + s) * L.q_sf_bytes;
+              for (int a = 0; a < atoms; ++a)
+                tmem_cp_32x128b_x4(
+                    tmem_base + sfb_col0 + (qb.idx * kNSUB + s) * 4 * atoms + 4 * a,
+                    sdesc_rows16_noswizzle(smem_u32(sf + sf_raw_bytes_q(n_cols) + 512 * a)));
+            }
+            mma_commit(sfq_ready + qb.idx);
+            last_commit = sfq_ready + qb.idx;
+            last_commit_phase = qb.phase;
+          }
+          __syncwarp();
+          new_q = false;
+        }
+        if (!mbar_wait(full_k + st.idx, st.phase, ctl, 17)) break;
+        for (int i = 0; i < g; ++i) {
+          uint8_t *sf = sksf + (st.idx * kG + i) * L.k_sf_bytes;
+          const int r = (c.q.y0 + (c.j + i) * kBlockM) & (kSfPad - 1);
+          sf_reorder_atom(reinterpret_cast<const uint32_t *>(sf) + r, 128,
+                          reinterpret_cast<uint32_t *>(sf + kSfRawBytesK));
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tc_fence_after_sync();
+          for (int i = 0; i < g; ++i)
+            tmem_cp_32x128b_x4(tmem_base + sfa_col0 + (st.idx * kG + i) * 4,
+                               sdesc_rows16_noswizzle(smem_u32(
+                                   sksf + (st.idx * kG + i) * L.k_sf_bytes + kSfRawBytesK)));
+          mma_commit(sf_ready + st.idx);
+          last_commit = sf_ready + st.idx;
+          last_commit_phase = st.phase;
+        }
+        __syncwarp();
+        st.next(kSTAGES);
+        if (cursor_step(P, tqt, c, g) && c.left > 0) {
+          qb.next(kQBUF);
+          new_q = true;
+        }
+      }
+      // copies still in flight must land before TMEM is released
+      if (lane == 0 && last_commit) mbar_drain(last_commit, last_commit_phase, p.wait_limit_ns);
+      __syncwarp();
+    }
+  } else if (warp < 2 + kEPI) {
     // ---------------- epilogue ----------------
     const int epi = warp - 2;                  // 0 .. kEPI-1
     const int quad = warp & 3;                 // TMEM lane quadrant of this warp
@@ -750,76 +860,83 @@ __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
     }
     if (R.a_count > 0) {
       Ring ac;
-      QBlk q;
-      int j = R.a_j;
-      make_qb(P, tqt, R.a_seq, R.a_b, R.a_seqoff, q);
-      bool ok = true;
-      // H=64: this warp's w rows for the current query block (warp-private)
+      ItemCursor c;
+      cursor_start(P, tqt, R, c);
+      bool ok = true, new_q = true;
+      int nsub = 1;
+      // H=64: this warp's w rows for the current query block (warp-private).
+      // kG == 1: the warp groups split each sub-block's tokens; kG > 1: they
+      // split the item's tiles, and every group takes all tokens.
       float *wrows = reinterpret_cast<float *>(smem + L.off_w) + epi * kWRowsPerWarp * 64;
-      int w_seq = -1, w_b = -1;
-      for (int64_t n = 0; n < R.a_count && ok; ++n) {
-        const int nsub = (q.ntok + p.tq_sub - 1) / p.tq_sub;
-        if constexpr (kH == 64) {
-          if (q.b != w_b || q.seq != w_seq) {
-            w_b = q.b;
-            w_seq = q.seq;
-            const int per = (p.tq_sub + kGroups - 1) / kGroups;
+      const int per = kG > 1 ? p.tq_sub : (p.tq_sub + kGroups - 1) / kGroups;
+      while (c.left > 0 && ok) {
+        const int g = cursor_tiles<kG>(c);
+        const QBlk &q = c.q;
+        if (new_q) {
+          nsub = (q.ntok + p.tq_sub - 1) / p.tq_sub;
+          if constexpr (kH == 64) {
             __syncwarp();
             for (int s = 0; s < nsub; ++s) {
               const int ntok_s = min(p.tq_sub, q.ntok - s * p.tq_sub);
-              const int i_lo = min(ntok_s, group * per), i_hi = min(ntok_s, i_lo + per);
+              const int i_lo = kG > 1 ? 0 : min(ntok_s, group * per);
+              const int i_hi = kG > 1 ? ntok_s : min(ntok_s, i_lo + per);
               for (int idx = lane; idx < (i_hi - i_lo) * 16; idx += 32) {
-                const int u = idx / 16, c = idx % 16;
+                const int u = idx / 16, cc = idx % 16;
                 const int t = q.t0 + s * p.tq_sub + i_lo + u;
-                reinterpret_cast<float4 *>(wrows + (s * per + u) * 64)[c] =
-                    __ldg(reinterpret_cast<const float4 *>(p.w + static_cast<int64_t>(t) * 64) + c);
+                reinterpret_cast<float4 *>(wrows + (s * per + u) * 64)[cc] =
+                    __ldg(reinterpret_cast<const float4 *>(p.w + static_cast<int64_t>(t) * 64) + cc);
               }
             }
             __syncwarp();
           }
+          new_q = false;
         }
-        const int64_t slot = static_cast<int64_t>(j) * kBlockM + quad * 32 + lane;
-        const bool in_row = slot < q.row_len;
-        for (int s = 0; s < nsub; ++s) {
+        const int nslots = kG > 1 ? 1 : nsub;
+        for (int s = 0; s < nslots; ++s) {
           if (!mbar_wait(acc_full + ac.idx, ac.phase, ctl, 22)) { ok = false; break; }
           tc_fence_after_sync();
-          const uint32_t tbase = tmem_base + lane_addr + ac.idx * n_cols;
-          const int i0 = s * p.tq_sub;
+          const int sub = kG > 1 ? 0 : s;
+          const int i0 = sub * p.tq_sub;
           const int ntok_s = min(p.tq_sub, q.ntok - i0);
-          if constexpr (kH == 64) {
-            // this warp's tokens of the sub-block: adjacent pair (or one)
-            const int per = (p.tq_sub + kGroups - 1) / kGroups;
-            const int i_lo = min(ntok_s, group * per), i_hi = min(ntok_s, i_lo + per);
-            const float *wsh = wrows + (s * per) * 64;
-            {
+          const int nacc = kG > 1 ? g : 1;
+          for (int a = 0; a < nacc; ++a) {
+            if (kG > 1 && kGroups > 1 && a % kGroups != group) continue;
+            const int64_t slot = static_cast<int64_t>(c.j + a) * kBlockM + quad * 32 + lane;
+            const bool in_row = slot < q.row_len;
+            const uint32_t tbase = tmem_base + lane_addr + (ac.idx * kAPS + a) * n_cols;
+            if constexpr (kH == 64) {
+              // this warp's tokens of the sub-block: adjacent pair (or one)
+              const int i_lo = kG > 1 ? 0 : min(ntok_s, group * per);
+              const int i_hi = kG > 1 ? ntok_s : min(ntok_s, i_lo + per);
+              const float *wsh = wrows + (sub * per) * 64;
               for (int i = i_lo; i < i_hi; ++i) {
                 const float acc = head_sum_h64(tbase + i * 64, wsh + (i - i_lo) * 64);
                 const int lv = qb_last_valid(P, q, i0 + i);
                 if (in_row)
                   p.scores[q.out0 + (i0 + i) * q.row_len + slot] = slot <= lv ? acc : kMaskBound;
               }
-            }
-          } else {
-            // any H: walk the sub-block's columns in 16-wide chunks
-            const int H = p.H, ncols = ntok_s * H;
-            const float *wsub = p.w + static_cast<int64_t>(q.t0 + i0) * H;
-            float acc = 0.f;
-            int tok = 0, h = 0;
-            for (int c0 = 0; c0 < ncols; c0 += 16) {
-              float v[16];
-              tmem_ld16_wait(tbase + c0, v);
+            } else {
+              // any H: walk the sub-block's columns in 16-wide chunks
+              const int H = p.H, ncols = ntok_s * H;
+              const float *wsub = p.w + static_cast<int64_t>(q.t0 + i0) * H;
+              float acc = 0.f;
+              int tok = 0, h = 0;
+              for (int c0 = 0; c0 < ncols; c0 += 16) {
+                float v[16];
+                tmem_ld16_wait(tbase + c0, v);
 #pragma unroll
-              for (int c = 0; c < 16; ++c) {
-                if (c0 + c < ncols) {
-                  acc = fmaf(__ldg(wsub + c0 + c), fmaxf(v[c], 0.f), acc);
-                  if (++h == H) {
-                    const int lv = qb_last_valid(P, q, i0 + tok);
-                    if (in_row)
-                      p.scores[q.out0 + (i0 + tok) * q.row_len + slot] =
-                          slot <= lv ? acc : kMaskBound;
-                    acc = 0.f;
-                    h = 0;
-                    ++tok;
+                for (int cc = 0; cc < 16; ++cc) {
+                  if (c0 + cc < ncols) {
+                    acc = fmaf(__ldg(wsub + c0 + cc), fmaxf(v[cc], 0.f), acc);
+                    if (++h == H) {
+                      const int lv = qb_last_valid(P, q, i0 + tok);
+                      if (in_row)
+                        p.scores[q.out0 + (i0 + tok) * q.row_len + slot] =
+                            slot <= lv ? acc : kMaskBound;
+                      acc = 0.f;
+                      h = 0;
+                      ++tok;
+                    }
                   }
                 }
               }
@@ -830,7 +947,7 @@ __global__ void __launch_bounds__((2 + kEPI) * 32, 1)
           if (lane == 0) mbar_arrive(acc_empty + ac.idx);
           ac.next(kNACC);
         }
-        if (ok && n + 1 < R.a_count) next_active(P, tqt, q, j);
+        if (ok && cursor_step(P, tqt, c, g)) new_q = true;
       }
     }
   }

@@ -431,21 +431,26 @@ __device__ __forceinline__ bool cursor_step(const ScoreParams &p, int tqt, ItemC
 
 // One token with H == 64 (the tuned head count): one load of the 64 TMEM
 // columns (heads 0..63 of this slot), w row from shared memory, four
-// independent partial sums.
+// independent partial sums (heads h = 4i + r into sum r), accumulated two at
+// a time with packed fp32 FMAs.
 __device__ __forceinline__ float head_sum_h64(uint32_t taddr, const float *wrow) {
   uint32_t r[64];
   tmem_ld64_wait(taddr, r);
   const float4 *w4 = reinterpret_cast<const float4 *>(wrow);
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const float4 wv = w4[i];
-    a0 = fmaf(wv.x, fmaxf(__uint_as_float(r[4 * i + 0]), 0.f), a0);
-    a1 = fmaf(wv.y, fmaxf(__uint_as_float(r[4 * i + 1]), 0.f), a1);
-    a2 = fmaf(wv.z, fmaxf(__uint_as_float(r[4 * i + 2]), 0.f), a2);
-    a3 = fmaf(wv.w, fmaxf(__uint_as_float(r[4 * i + 3]), 0.f), a3);
+    a01 = ffma2(make_float2(wv.x, wv.y),
+                make_float2(fmaxf(__uint_as_float(r[4 * i + 0]), 0.f),
+                            fmaxf(__uint_as_float(r[4 * i + 1]), 0.f)),
+                a01);
+    a23 = ffma2(make_float2(wv.z, wv.w),
+                make_float2(fmaxf(__uint_as_float(r[4 * i + 2]), 0.f),
+                            fmaxf(__uint_as_float(r[4 * i + 3]), 0.f)),
+                a23);
   }
-  return (a0 + a1) + (a2 + a3);
+  return (a01.x + a01.y) + (a23.x + a23.y);
 }
 
 __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
@@ -510,7 +515,7 @@ __global__ void __launch_bounds__((2 + kEPI + (kFP8 ? 1 : 0) + (kISS - 1)) * 32,
                  const __grid_constant__ CUtensorMap tmap_ksf,
                  const __grid_constant__ CUtensorMap tmap_qsf,
                  const ScoreParams p) {
-  static_assert(kEPI == 4 || kEPI == 8, "epilogue warps");
+  static_assert(kEPI == 4 || kEPI == 8 || kEPI == 16, "epilogue warps");
   static_assert(kH == 64 || kEPI == 4, "generic epilogue uses 4 warps");
   static_assert(kG == 1 || kNSUB == 1, "tile batching is for single sub-block queries");
   static_assert(kISS == 1 || kISS == 2, "issuers");

@@ -504,7 +504,7 @@ def main(argv=None):
         roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
                 "frac": achieved / pk["hbm"]}
     traffic = profiled_traffic(wl.name)
-    roof.update(traffic=traffic, kernel="score_bf16_kernel",
+    roof.update(traffic=traffic, kernel="score_kernel",
                 kernel_ms=r["ms_score"], peak_source=f"{pk['src']} (MEASURED_PEAKS.json)"
                 if pk["src"] == "measured" else "fallback")
     t_roof = max(r["flops"] / (pk["bf16"] * (2.0 if wl.dtype == syn.DTYPE_FP8 else 1.0) * 1e12),

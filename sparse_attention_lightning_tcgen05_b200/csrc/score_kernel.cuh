@@ -429,28 +429,43 @@ __device__ __forceinline__ bool cursor_step(const ScoreParams &p, int tqt, ItemC
 
 // ---- epilogue helpers ---------------------------------------------------------------
 
-// One token with H == 64 (the tuned head count): one load of the 64 TMEM
-// columns (heads 0..63 of this slot), w row from shared memory, four
-// independent partial sums (heads h = 4i + r into sum r), accumulated two at
-// a time with packed fp32 FMAs.
+// One token with H == 64 (the tuned head count): heads 0..63 of this slot
+// from TMEM in two 32-column halves, the w row from shared memory, eight
+// independent partial sums (heads h = 32j + 4i + r into sum 4j + r, in four
+// packed pairs), so that the packed fp32 FMAs form four short dependency
+// chains instead of two long ones. The w loads of each half are issued
+// before the TMEM load they pair with, so their latency is hidden behind it.
 __device__ __forceinline__ float head_sum_h64(uint32_t taddr, const float *wrow) {
-  uint32_t r[64];
-  tmem_ld64_wait(taddr, r);
   const float4 *w4 = reinterpret_cast<const float4 *>(wrow);
-  float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                   make_float2(0.f, 0.f)};
+  float4 wv[8];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const float4 wv = w4[i];
-    a01 = ffma2(make_float2(wv.x, wv.y),
-                make_float2(fmaxf(__uint_as_float(r[4 * i + 0]), 0.f),
-                            fmaxf(__uint_as_float(r[4 * i + 1]), 0.f)),
-                a01);
-    a23 = ffma2(make_float2(wv.z, wv.w),
-                make_float2(fmaxf(__uint_as_float(r[4 * i + 2]), 0.f),
-                            fmaxf(__uint_as_float(r[4 * i + 3]), 0.f)),
-                a23);
+  for (int i = 0; i < 8; ++i) wv[i] = w4[i];
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    float r[32];
+    tmem_ld32_wait(taddr + 32 * half, r);
+    float4 wn[8];
+    if (half == 0) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) wn[i] = w4[8 + i];
+    }
+    float2 &p01 = acc[2 * half], &p23 = acc[2 * half + 1];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      p01 = ffma2(make_float2(wv[i].x, wv[i].y),
+                  make_float2(fmaxf(r[4 * i + 0], 0.f), fmaxf(r[4 * i + 1], 0.f)), p01);
+      p23 = ffma2(make_float2(wv[i].z, wv[i].w),
+                  make_float2(fmaxf(r[4 * i + 2], 0.f), fmaxf(r[4 * i + 3], 0.f)), p23);
+    }
+    if (half == 0) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) wv[i] = wn[i];
+    }
   }
-  return (a01.x + a01.y) + (a23.x + a23.y);
+  return ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
+         ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
 }
 
 __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }

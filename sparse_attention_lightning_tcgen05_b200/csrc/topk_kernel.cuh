@@ -57,6 +57,7 @@ struct TopkShared {
   uint32_t out_gt, out_eq;       // output cursors of the unordered pass
   uint32_t tie_idx[32];          // slots of the ties (when at most 32)
   uint32_t small[32];            // the last <= 32 candidates
+  uint32_t nsmall;
   int seq;
   long long seq_off;
   // followed by the staged keys (dynamic size)
@@ -376,32 +377,29 @@ __global__ void __launch_bounds__(NT) topk_kernel(const TopkParams p) {
   }
   if (lo_bit > 0) {
     // <= 32 candidates share the prefix: the need-th largest of them, by
-    // counting for each candidate the ones above it (one warp, no barrier).
-    if (tid < 32) {
-      // compact the candidates that share the prefix into sm.small (the list
-      // may still hold keys compacted under a shorter prefix)
-      const uint32_t nc = sm.ncand;
-      uint32_t filled = 0;
-      for (uint32_t c0 = 0; c0 < nc; c0 += 32) {
-        const uint32_t i = c0 + tid;
-        const uint32_t key = i < nc ? sm.cand[i] : 0u;
-        const bool m = i < nc && ((key - kmin) >> lo_bit) == prefix;
-        const unsigned mm = __ballot_sync(0xffffffffu, m);
-        const uint32_t slot = filled + __popc(mm & ((1u << tid) - 1u));
-        if (m && slot < 32) sm.small[slot] = key;
-        filled += __popc(mm);
+    // counting for each candidate the ones above it. The block collects them
+    // (the list may still hold keys compacted under a shorter prefix), then
+    // one warp ranks them.
+    if (tid == 0) sm.nsmall = 0;
+    __syncthreads();
+    const uint32_t nc = sm.ncand;
+    for (uint32_t i = tid; i < nc; i += NT) {
+      const uint32_t key = sm.cand[i];
+      if (((key - kmin) >> lo_bit) == prefix) {
+        const uint32_t slot = atomicAdd(&sm.nsmall, 1u);
+        if (slot < 32) sm.small[slot] = key;
       }
-      __syncwarp();
-      const bool live = static_cast<uint32_t>(tid) < min(filled, 32u);
+    }
+    __syncthreads();
+    if (tid < 32) {
+      const uint32_t live_n = min(sm.nsmall, 32u);
+      const bool live = static_cast<uint32_t>(tid) < live_n;
       const uint32_t mine = live ? sm.small[tid] : 0u;
       uint32_t above = 0, equal = 0;
-      for (int l = 0; l < 32; ++l) {
-        const uint32_t other = __shfl_sync(0xffffffffu, mine, l);
-        const bool other_live = __shfl_sync(0xffffffffu, live ? 1 : 0, l) != 0;
-        if (other_live) {
-          above += other > mine;
-          equal += other == mine;
-        }
+      for (uint32_t l = 0; l < live_n; ++l) {
+        const uint32_t other = sm.small[l];
+        above += other > mine;
+        equal += other == mine;
       }
       const bool is_tau = live && above < need && need <= above + equal;
       const unsigned who = __ballot_sync(0xffffffffu, is_tau);

@@ -41,8 +41,12 @@ constexpr int kClusterCand = 1024;     // candidates every rank gathers
 
 template <int NT>
 struct ClusterTopkShared {
-  alignas(16) uint32_t hist[2][kClusterBins];                 // this CTA's, by round parity
-  alignas(16) uint32_t part[kClusterMaxRanks][kClusterBins];  // every rank's, this round
+  alignas(16) uint32_t hist[2][kClusterBins];                 // this CTA's (hist[0] reused)
+  // every rank's histogram of the round, pushed here by its owner before the
+  // round's barrier; by round parity, so that a rank already pushing the
+  // next round never overwrites one still being read
+  alignas(16) uint32_t part[2][kClusterMaxRanks][kClusterBins];
+  uint32_t rk_min[kClusterMaxRanks], rk_max[kClusterMaxRanks];  // pushed key ranges
   uint32_t ghist[kClusterBins];                               // their sum
   uint32_t cand[kClusterCand];          // the candidates of all ranks, rank by rank
   uint32_t gt_above[kClusterMaxRanks];  // per rank: keys above the selected bins
@@ -229,13 +233,20 @@ __global__ void __launch_bounds__(NT) topk_cluster_kernel(const TopkParams p) {
   }
 
   // ---- 1. stage the chunk; the row's key range (barrier A) ----
+  // Exchanges push: each rank stores its data into every rank's shared
+  // memory before the barrier (the barrier's release/acquire makes it
+  // visible), so nothing waits on a remote load after it.
   stage_keys<NT>(row + lo, m, staged ? staged_keys : nullptr, sm);
+  if (static_cast<uint32_t>(tid) < C) {
+    dsmem_st(dsmem_addr(smem_u32(&sm.rk_min[r]), tid), sm.kmin);
+    dsmem_st(dsmem_addr(smem_u32(&sm.rk_max[r]), tid), sm.kmax);
+  }
   cluster_sync();
   if (tid < 32) {
     uint32_t a = 0xffffffffu, b = 0u;
     if (static_cast<uint32_t>(lane) < C) {
-      a = dsmem_ld(dsmem_addr(smem_u32(&sm.kmin), lane));
-      b = dsmem_ld(dsmem_addr(smem_u32(&sm.kmax), lane));
+      a = sm.rk_min[lane];
+      b = sm.rk_max[lane];
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
@@ -269,7 +280,7 @@ __global__ void __launch_bounds__(NT) topk_cluster_kernel(const TopkParams p) {
     const int dbits = value_round ? 8 : (lo_bit >= 8 ? 8 : lo_bit);
     const int shift = value_round ? 0 : lo_bit - dbits;
     const uint32_t dmask = (1u << dbits) - 1u;
-    uint32_t *h = sm.hist[buf];
+    uint32_t *h = sm.hist[0];
     for (int b = tid; b < kClusterBins; b += NT) h[b] = 0;
     __syncthreads();
     for (uint32_t i = tid; i < m; i += NT) {
@@ -280,16 +291,16 @@ __global__ void __launch_bounds__(NT) topk_cluster_kernel(const TopkParams p) {
                   1u);
     }
     __syncthreads();
-    cluster_sync();
-    if (static_cast<uint32_t>(tid) < 64u * C) {   // copy every rank's histogram
-      const int src = tid >> 6, q = tid & 63;
-      *reinterpret_cast<uint4 *>(&sm.part[src][4 * q]) =
-          dsmem_ld4(dsmem_addr(smem_u32(&h[4 * q]), src));
+    uint32_t (*part)[kClusterBins] = sm.part[buf];
+    if (static_cast<uint32_t>(tid) < 64u * C) {   // push this histogram to every rank
+      const int dst = tid >> 6, q = tid & 63;
+      dsmem_st4(dsmem_addr(smem_u32(&part[r][4 * q]), dst),
+                *reinterpret_cast<const uint4 *>(&h[4 * q]));
     }
-    __syncthreads();
+    cluster_sync();
     if (tid < kClusterBins) {
       uint32_t sum = 0;
-      for (uint32_t j = 0; j < C; ++j) sum += sm.part[j][tid];
+      for (uint32_t j = 0; j < C; ++j) sum += part[j][tid];
       sm.ghist[tid] = sum;
     }
     __syncthreads();
@@ -297,11 +308,11 @@ __global__ void __launch_bounds__(NT) topk_cluster_kernel(const TopkParams p) {
     const uint32_t bin = sm.sel_bin;
     if (static_cast<uint32_t>(warp) < C) {        // per rank: above the bin, in it
       uint32_t above = 0;
-      for (int b = static_cast<int>(bin) + 1 + lane; b < (1 << dbits); b += 32) above += sm.part[warp][b];
+      for (int b = static_cast<int>(bin) + 1 + lane; b < (1 << dbits); b += 32) above += part[warp][b];
       above = __reduce_add_sync(0xffffffffu, above);
       if (lane == 0) {
         sm.gt_above[warp] += above;
-        sm.cnt_sel[warp] = sm.part[warp][bin];
+        sm.cnt_sel[warp] = part[warp][bin];
       }
     }
     __syncthreads();

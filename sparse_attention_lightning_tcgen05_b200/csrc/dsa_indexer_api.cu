@@ -190,33 +190,50 @@ int pow2_floor(int x) {
 
 // Kernel instances. Decode with one cache per token (H = 64): two key tiles
 // per pipeline item. Prefill / a shared cache (H = 64): 8 tokens per query
-// block as two N = 256 sub-blocks. Any other H: the generic epilogue.
+// block as two N = 256 sub-blocks. Any other H: the generic epilogue. Each
+// instance is compiled for one mask mode.
+constexpr int kPos = dsa::kModePositions, kCau = dsa::kModeCausal;
+
 ScoreLaunch choose_score(const dsa_indexer_desc_t *d) {
-  const bool per_token_cache = d->mask == DSA_MASK_POSITIONS && d->k_seq_stride != 0;
+  const bool causal = d->mask == DSA_MASK_CAUSAL;
+  const bool per_token_cache = !causal && d->k_seq_stride != 0;
   const int H = d->H;
   if (d->dtype == DSA_KV_BF16) {
     if (per_token_cache) {
       if (H == 64)
-        return {dsa::score_kernel<64, 1, 2, 3, 2, 2, 8, false, 2>, 0, 2, 2, 1, 8, 2, 2, 1, 64, 64, false};
-      return {dsa::score_kernel<0, 1, 1, 2, 4, 1, 4, false, 1>, 1, 4, 1, 1, 4, 1, 1, 1, round16(H), 256,
-              false};
+        return {dsa::score_kernel<64, 1, 2, 3, 2, 2, 8, false, 2, kPos>, 0, 2, 2, 1, 8, 2, 2, 1, 64,
+                64, false};
+      return {dsa::score_kernel<0, 1, 1, 2, 4, 1, 4, false, 1, kPos>, 1, 4, 1, 1, 4, 1, 1, 1,
+              round16(H), 256, false};
     }
     if (H == 64)
-      return {dsa::score_kernel<64, 2, 1, 2, 2, 1, 8, false, 1>, 2, 2, 1, 2, 8, 1, 1, 4, 256, 256, false};
+      return causal ? ScoreLaunch{dsa::score_kernel<64, 2, 1, 2, 2, 1, 8, false, 1, kCau>, 2, 2, 1,
+                                  2, 8, 1, 1, 4, 256, 256, false}
+                    : ScoreLaunch{dsa::score_kernel<64, 2, 1, 2, 2, 1, 8, false, 1, kPos>, 6, 2, 1,
+                                  2, 8, 1, 1, 4, 256, 256, false};
     const int tq = pow2_floor(std::min(128, 256 / H));
-    return {dsa::score_kernel<0, 1, 1, 2, 4, 1, 4, false, 1>, 1, 4, 1, 1, 4, 1, 1, tq, round16(tq * H),
-            256, false};
+    return causal ? ScoreLaunch{dsa::score_kernel<0, 1, 1, 2, 4, 1, 4, false, 1, kCau>, 7, 4, 1, 1,
+                                4, 1, 1, tq, round16(tq * H), 256, false}
+                  : ScoreLaunch{dsa::score_kernel<0, 1, 1, 2, 4, 1, 4, false, 1, kPos>, 1, 4, 1, 1,
+                                4, 1, 1, tq, round16(tq * H), 256, false};
   }
   if (per_token_cache) {
     if (H == 64)
-      return {dsa::score_kernel<64, 1, 2, 3, 5, 2, 8, true, 2>, 3, 5, 2, 1, 8, 2, 2, 1, 64, 64, true};
-    return {dsa::score_kernel<0, 1, 1, 2, 4, 1, 4, true, 1>, 4, 4, 1, 1, 4, 1, 1, 1, round16(H), 128, true};
+      return {dsa::score_kernel<64, 1, 2, 3, 5, 2, 8, true, 2, kPos>, 3, 5, 2, 1, 8, 2, 2, 1, 64,
+              64, true};
+    return {dsa::score_kernel<0, 1, 1, 2, 4, 1, 4, true, 1, kPos>, 4, 4, 1, 1, 4, 1, 1, 1,
+            round16(H), 128, true};
   }
   if (H == 64)
-    return {dsa::score_kernel<64, 2, 1, 2, 4, 1, 8, true, 1>, 5, 4, 1, 2, 8, 1, 1, 2, 128, 128, true};
+    return causal ? ScoreLaunch{dsa::score_kernel<64, 2, 1, 2, 4, 1, 8, true, 1, kCau>, 5, 4, 1, 2,
+                                8, 1, 1, 2, 128, 128, true}
+                  : ScoreLaunch{dsa::score_kernel<64, 2, 1, 2, 4, 1, 8, true, 1, kPos>, 10, 4, 1,
+                                2, 8, 1, 1, 2, 128, 128, true};
   const int tq = pow2_floor(std::min(128, 128 / H));
-  return {dsa::score_kernel<0, 1, 1, 2, 4, 1, 4, true, 1>, 4, 4, 1, 1, 4, 1, 1, tq, round16(tq * H), 128,
-          true};
+  return causal ? ScoreLaunch{dsa::score_kernel<0, 1, 1, 2, 4, 1, 4, true, 1, kCau>, 11, 4, 1, 1, 4,
+                              1, 1, tq, round16(tq * H), 128, true}
+                : ScoreLaunch{dsa::score_kernel<0, 1, 1, 2, 4, 1, 4, true, 1, kPos>, 4, 4, 1, 1, 4,
+                              1, 1, tq, round16(tq * H), 128, true};
 }
 
 dsa_status_t launch_score(const dsa_indexer_desc_t *d, const void *q, const uint8_t *q_scale,

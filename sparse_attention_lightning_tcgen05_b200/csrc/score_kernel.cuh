@@ -519,11 +519,13 @@ __device__ __forceinline__ void sf_reorder_atom(const uint32_t *rows, int nrows,
 // kFP8: e4m3 + e8m0/32 inputs through the block-scaled MMA.
 // kISS: MMA-issuing warps (1 or 2). With 2, items alternate between them so
 //     that one warp's waits and commits overlap the other's MMAs.
+// kMODE: kModePositions or kModeCausal, fixed at compile time so that each
+//     instance carries only its own schedule code.
 //
 // Warps: 0 TMA producer, 1 MMA issuer (+ TMEM owner), 2 .. 1+kEPI epilogue,
 // then (fp8) the scale-factor warp, then (kISS == 2) the second issuer.
 template <int kH, int kNSUB, int kG, int kNACC, int kSTAGES, int kQBUF, int kEPI, bool kFP8,
-          int kISS>
+          int kISS, int kMODE>
 __global__ void __launch_bounds__((2 + kEPI + (kFP8 ? 1 : 0) + (kISS - 1)) * 32, 1)
     score_kernel(const __grid_constant__ CUtensorMap tmap_k,
                  const __grid_constant__ CUtensorMap tmap_q,
@@ -598,11 +600,12 @@ __global__ void __launch_bounds__((2 + kEPI + (kFP8 ? 1 : 0) + (kISS - 1)) * 32,
 
   // Decode positions are read by every role many times: keep a copy here.
   int *spos = reinterpret_cast<int *>(smem + L.off_pos);
-  const bool pos_staged = p.mode == kModePositions && p.T <= kPosCap;
+  const bool pos_staged = kMODE == kModePositions && p.T <= kPosCap;
   if (pos_staged)
     for (int i = threadIdx.x; i < p.T; i += blockDim.x) spos[i] = __ldg(p.positions + i);
   __syncthreads();
   ScoreParams P = p;
+  P.mode = kMODE;   // a constant from here on: the other mode's code folds away
   if (pos_staged) P.positions = spos;
   if (warp == 0) {
     CtaRange R;

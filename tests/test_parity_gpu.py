@@ -80,6 +80,13 @@ def test_decode_position_edges(dsa):
     run_and_check(dsa, wl, inputs)
 
 
+def test_decode_many_tokens(dsa):
+    """More than 32 query blocks (the positions schedule scans blocks 32 at a
+    time) and pipeline items of two key tiles that end at token boundaries."""
+    wl = decode_wl(T=100, H=64, S=1000, k=64, pos=(0, 1000), seed=40)
+    run_and_check(dsa, wl, syn.generate(wl))
+
+
 def test_decode_shared_cache(dsa):
     wl = decode_wl(T=11, H=64, S=900, k=50, shared=True, pos=(0, 900), seed=6)
     run_and_check(dsa, wl, syn.generate(wl))
@@ -182,3 +189,8 @@ def test_long_decode_fp8_full_size_sampled(dsa):
     rng = np.random.default_rng(13)
     rows = sorted(set([0, 1, 63] + list(rng.integers(0, wl.T, 5))))
     run_and_check(dsa, wl, syn.generate(wl), rows=rows, tol=TOL_FP8)
+
+
+def test_fp8_decode_many_tokens(dsa):
+    wl = fp8_decode_wl(T=70, H=64, S=1300, k=80, pos=(0, 1300), seed=41)
+    run_and_check(dsa, wl, syn.generate(wl), tol=TOL_FP8)

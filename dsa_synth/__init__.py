@@ -32,6 +32,7 @@ E4M3_MAX = 448.0         # largest finite e4m3 magnitude
 
 MODE_POSITIONS = 0       # decode: slot s valid iff s <= positions[t]
 MODE_CAUSAL = 1          # packed prefill: slot s valid iff s <= t (sequence-local)
+MODE_COMPRESSED = 2      # pooled (C4) keys: slot j valid iff (j+1)*r <= query_start+t+1
 DTYPE_BF16 = 0
 DTYPE_FP8 = 1
 
@@ -40,24 +41,28 @@ DTYPE_FP8 = 1
 class Workload:
     """One synthetic indexer problem (sizes, mask rule, value distributions)."""
     name: str
-    mode: int                      # MODE_POSITIONS or MODE_CAUSAL
+    mode: int                      # MODE_POSITIONS, MODE_CAUSAL or MODE_COMPRESSED
     T: int                         # query tokens
     H: int                         # indexer heads
     D: int                         # head_dim
     index_topk: int
     dtype: int = DTYPE_BF16
-    S: int = 0                     # POSITIONS: slots per sequence cache
+    S: int = 0                     # POSITIONS: slots per sequence cache; COMPRESSED: pooled slots
     shared_cache: bool = False     # POSITIONS: one cache for every token
     pos_lo: int = 0                # POSITIONS: positions ~ U[pos_lo, pos_hi)
     pos_hi: int = 0
     seqlens: tuple = ()            # CAUSAL: packed sequence lengths
     w_scale: float = 1.0
     seed: int = 0
+    query_start: int = 0           # COMPRESSED: absolute position of query 0
+    compress_ratio: int = 0        # COMPRESSED: tokens pooled per slot
 
     @property
     def num_seqs(self) -> int:
         if self.mode == MODE_CAUSAL:
             return len(self.seqlens)
+        if self.mode == MODE_COMPRESSED:
+            return 1
         return 1 if self.shared_cache else self.T
 
     @property
@@ -70,7 +75,7 @@ class Workload:
     @property
     def k_seq_stride(self) -> int:
         """Elements between consecutive sequences' caches (POSITIONS)."""
-        if self.mode == MODE_CAUSAL or self.shared_cache:
+        if self.mode != MODE_POSITIONS or self.shared_cache:
             return 0
         return self.S * self.D
 
@@ -98,6 +103,11 @@ WORKLOADS = {
                                D=128, index_topk=2048,
                                seqlens=(4096, 16384, 32768, 65536),
                                w_scale=1.0 / 8.0),
+    # compressed (C4) indexer, the next step beyond the five: an 8192-token
+    # prefill chunk against its 2048 keys pooled 4:1, DSV4's index_topk 1024
+    "c4_prefill": Workload("c4_prefill", MODE_COMPRESSED, T=8192, H=64, D=128,
+                           index_topk=1024, S=2048, compress_ratio=4,
+                           query_start=0, w_scale=1.0 / 8.0),
 }
 
 
@@ -208,7 +218,8 @@ def generate(wl: Workload, value_kind: str = "gauss",
     Keys of the returned dict: q ([T,H,D] uint16 bf16 bits or uint8 e4m3),
     q_scale ([T,H,D/32] uint8 or None), k ([key_slots, D]), k_scale, w
     ([T,H] float32), positions ([T] int32, POSITIONS only), cu_seqlens
-    ([num_seqs+1] int32, CAUSAL only).
+    ([num_seqs+1] int32, CAUSAL only). COMPRESSED draws neither: validity
+    follows from query_start and compress_ratio.
     """
     rng = np.random.default_rng(wl.seed if seed is None else seed)
     T, H, D = wl.T, wl.H, wl.D
@@ -227,6 +238,6 @@ def generate(wl: Workload, value_kind: str = "gauss",
     if wl.mode == MODE_POSITIONS:
         out["positions"] = rng.integers(wl.pos_lo, wl.pos_hi, size=T,
                                         dtype=np.int32)
-    else:
+    elif wl.mode == MODE_CAUSAL:
         out["cu_seqlens"] = wl.cu_seqlens()
     return out

@@ -44,7 +44,8 @@ class _Problem(ctypes.Structure):
                 ("positions", ctypes.c_void_p), ("cu_seqlens", ctypes.c_void_p),
                 ("q", ctypes.c_void_p), ("q_scale", ctypes.c_void_p),
                 ("w", ctypes.c_void_p), ("k", ctypes.c_void_p),
-                ("k_scale", ctypes.c_void_p)]
+                ("k_scale", ctypes.c_void_p), ("query_start", ctypes.c_int64),
+                ("compress_ratio", ctypes.c_int32), ("pad_", ctypes.c_int32)]
 
 
 _lib = None
@@ -101,7 +102,8 @@ class Problem:
             cu_seqlens=_ptr(a.get("cu_seqlens")),
             q=_ptr(a["q"]), q_scale=_ptr(a.get("q_scale")),
             w=_ptr(a["w"]),
-            k=_ptr(a["k"]), k_scale=_ptr(a.get("k_scale")))
+            k=_ptr(a["k"]), k_scale=_ptr(a.get("k_scale")),
+            query_start=wl.query_start, compress_ratio=wl.compress_ratio)
 
     def row_info(self, t: int):
         """(first_slot, row_len, last_valid, score_offset) of query row t."""

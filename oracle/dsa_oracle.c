@@ -28,6 +28,10 @@
  *    mathematical no-op for the score; scales are block-32 e8m0 (qr_scale_hbm).
  *  - NeMo AutoModel optimized_kernels, sparse_attention_torch parameters:
  *    a top-k index of -1 masks an entry.
+ *  - NeMo AutoModel optimized_kernels, dsv4_indexer_scores: the compressed
+ *    (C4) indexer scores queries against pooled_kv, keys pooled over
+ *    compress_ratio consecutive tokens, for a query chunk that starts at
+ *    absolute position query_start.
  *  - The head-weighted ReLU sum itself is the lightning-indexer definition
  *    that the pages name (lightning_indexer in the tokamax Supported Ops
  *    table: query-key relevance scores followed by top-k) but do not print;
@@ -36,6 +40,11 @@
  * Readings where the pages are silent:
  *  - valid(t,s) is inclusive: s <= positions[t] (decode) or s <= t within the
  *    row's sequence (causal prefill); the token's own key is at its position.
+ *  - Compressed mode: pooled slot j covers tokens [j*r, (j+1)*r) (r =
+ *    compress_ratio); query t sits at absolute position query_start + t and
+ *    sees slot j iff the whole block is at or before it: (j+1)*r <=
+ *    query_start + t + 1, i.e. j <= floor((query_start + t + 1) / r) - 1.
+ *    Every query scores the one pooled cache; rows are [T, S] like decode.
  *  - MASK_BOUND = -0x1.FEp127, the lowest finite bf16 value (exact in fp32).
  *  - Rows with fewer valid slots than index_topk select all valid slots and
  *    pad with -1; masked slots are never selected.
@@ -52,6 +61,7 @@
 
 #define ORC_MODE_POSITIONS 0
 #define ORC_MODE_CAUSAL 1
+#define ORC_MODE_COMPRESSED 2
 #define ORC_DTYPE_BF16 0
 #define ORC_DTYPE_FP8 1
 #define ORC_MX_BLOCK 32
@@ -60,7 +70,7 @@ static const double ORC_MASK_BOUND = -0x1.FEp127;
 
 /* The problem statement, as the pages give it (flat, host pointers). */
 typedef struct {
-    int32_t mode;            /* ORC_MODE_POSITIONS or ORC_MODE_CAUSAL */
+    int32_t mode;            /* ORC_MODE_POSITIONS, _CAUSAL or _COMPRESSED */
     int32_t dtype;           /* ORC_DTYPE_BF16 or ORC_DTYPE_FP8 (q and k) */
     int32_t T, H, D;
     int32_t num_seqs;        /* CAUSAL: packed sequences */
@@ -73,6 +83,9 @@ typedef struct {
     const float *w;             /* [T, H] */
     const void *k;              /* [slots, D] */
     const uint8_t *k_scale;     /* [slots, D/32] e8m0 (FP8) */
+    int64_t query_start;        /* COMPRESSED: absolute position of query 0 */
+    int32_t compress_ratio;     /* COMPRESSED: tokens pooled per slot (>= 1) */
+    int32_t pad_;
 } orc_problem;
 
 /* ---- exact decoding of the storage formats -------------------------------- */
@@ -137,6 +150,14 @@ int orc_row_info(const orc_problem *p, int64_t t, int64_t *first_slot,
         *first_slot = t * (p->k_seq_stride / p->D);
         *row_len = p->S;
         *last_valid = p->positions[t];          /* s <= positions[t] */
+        *score_offset = t * p->S;
+        return 0;
+    }
+    if (p->mode == ORC_MODE_COMPRESSED) {
+        *first_slot = 0;                        /* one pooled cache */
+        *row_len = p->S;
+        /* (j+1)*r <= query_start + t + 1 */
+        *last_valid = (p->query_start + t + 1) / p->compress_ratio - 1;
         *score_offset = t * p->S;
         return 0;
     }

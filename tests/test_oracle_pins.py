@@ -36,6 +36,12 @@ def _problem_from_golden(g):
                           index_topk=1, S=g["S"], shared_cache=True)
         inputs = dict(positions=np.asarray(g["positions"], np.int32),
                       cu_seqlens=None)
+    elif g["mode"] == "compressed":
+        wl = syn.Workload("golden", syn.MODE_COMPRESSED, T=T, H=H, D=D,
+                          index_topk=1, S=g["S"],
+                          compress_ratio=g["compress_ratio"],
+                          query_start=g["query_start"])
+        inputs = dict(positions=None, cu_seqlens=None)
     else:
         cu = g["cu_seqlens"]
         wl = syn.Workload("golden", syn.MODE_CAUSAL, T=T, H=H, D=D,
@@ -47,7 +53,8 @@ def _problem_from_golden(g):
     return wl, inputs
 
 
-@pytest.mark.parametrize("name", ["decode_hand.json", "causal_hand.json"])
+@pytest.mark.parametrize("name", ["decode_hand.json", "causal_hand.json",
+                                  "compressed_hand.json"])
 def test_golden_hand_worked(golden_dir, name):
     g = json.load(open(os.path.join(golden_dir, name)))
     wl, inputs = _problem_from_golden(g)
@@ -305,6 +312,60 @@ def test_shared_cache_rows_read_the_same_keys():
     inputs["positions"] = np.array([49, 20], np.int32)
     sc = oracle.Problem(wl, inputs).scores([0, 1])
     np.testing.assert_array_equal(sc[0][:21], sc[1][:21])
+
+
+def _small_compressed(T=40, H=3, S=23, r=4, qs=5, seed=4, dtype=syn.DTYPE_BF16):
+    wl = syn.Workload("c", syn.MODE_COMPRESSED, T=T, H=H, D=128, index_topk=8,
+                      S=S, compress_ratio=r, query_start=qs, dtype=dtype,
+                      w_scale=0.5, seed=seed)
+    return wl, syn.generate(wl)
+
+
+@pytest.mark.parametrize("r,qs", [(4, 0), (4, 5), (1, 0), (3, 17), (128, 100)])
+def test_compressed_visibility_by_raw_tokens(r, qs):
+    """A pooled slot is visible exactly when every raw token it pools sits at
+    or before the query's absolute position: enumerated token by token."""
+    wl, inputs = _small_compressed(T=50, S=30, r=r, qs=qs)
+    P = oracle.Problem(wl, inputs)
+    sc = P.scores(list(range(wl.T)))
+    for t in range(wl.T):
+        p = qs + t
+        vis = np.array([all(x <= p for x in range(j * r, (j + 1) * r))
+                        for j in range(wl.S)])
+        assert np.array_equal(sc[t] != MB, vis), (t, p)
+        first, L, last, off = P.row_info(t)
+        assert first == 0 and L == wl.S and off == t * wl.S
+        assert min(last, wl.S - 1) == int(vis.sum()) - 1   # unclamped, like a position
+
+
+@pytest.mark.parametrize("dtype", [syn.DTYPE_BF16, syn.DTYPE_FP8])
+def test_compressed_equals_shared_cache_positions(dtype):
+    """With every token reading the one pooled cache, the compressed rule is
+    the positions rule with position = the last fully pooled slot; rows that
+    see no slot are all at the mask bound and select nothing."""
+    wl, inputs = _small_compressed(T=37, S=19, r=4, qs=2, dtype=dtype)
+    rows = list(range(wl.T))
+    P = oracle.Problem(wl, inputs)
+    sc = P.scores(rows)
+    last = np.array([(wl.query_start + t + 1) // wl.compress_ratio - 1
+                     for t in rows])
+    wp = syn.Workload("p", syn.MODE_POSITIONS, T=wl.T, H=wl.H, D=wl.D,
+                      index_topk=8, S=wl.S, shared_cache=True, dtype=dtype)
+    ip = dict(inputs, positions=np.maximum(last, 0).astype(np.int32),
+              cu_seqlens=None)
+    sp = oracle.Problem(wp, ip).scores(rows)
+    for t in rows:
+        if last[t] < 0:
+            assert np.all(sc[t] == MB)
+        else:
+            np.testing.assert_array_equal(sc[t], sp[t])
+    for k in (1, 5, 19, 24):
+        tk = P.topk(rows, sc, k)
+        for t in rows:
+            n = max(0, min(k, int(last[t]) + 1))
+            got = tk[t].tolist()
+            assert got[n:] == [-1] * (k - n)
+            assert sorted(got[:n]) == sorted(_brute_topk(sc[t], int(last[t]), k)[:n])
 
 
 def test_causal_layout_tiles_packed_buffer():

@@ -44,20 +44,29 @@ DEFAULTS = {   # steps, warmup, graph length
     "long_decode_fp8": (6000, 300, 60),
     "prefill_causal": (1500, 30, 30),
     "ragged_prefill": (20, 3, 1),
+    "c4_prefill": (1500, 30, 30),
 }
 L2_BYTES = 126 * 2**20
 
 
 # ---------------------------------------------------------------- workload math
-def valid_pairs(wl, inputs) -> int:
+def row_positions(wl, inputs):
+    """Last valid slot of each row before clamping to the row (decode-style
+    rows): the token's position, or the last fully pooled slot."""
     if wl.mode == syn.MODE_POSITIONS:
-        p = np.asarray(inputs["positions"], np.int64)
-        return int(np.clip(p + 1, 0, wl.S).sum())
+        return np.asarray(inputs["positions"], np.int64)
+    t = np.arange(wl.T, dtype=np.int64)
+    return (wl.query_start + t + 1) // wl.compress_ratio - 1
+
+
+def valid_pairs(wl, inputs) -> int:
+    if wl.mode != syn.MODE_CAUSAL:
+        return int(np.clip(row_positions(wl, inputs) + 1, 0, wl.S).sum())
     return int(sum(L * (L + 1) // 2 for L in wl.seqlens))
 
 
 def score_elems(wl) -> int:
-    if wl.mode == syn.MODE_POSITIONS:
+    if wl.mode != syn.MODE_CAUSAL:
         return wl.T * wl.S
     return int(sum(L * L for L in wl.seqlens))
 
@@ -73,9 +82,10 @@ def algorithmic(wl, inputs):
     slot_bytes = wl.D * elt + (wl.D // 32 if wl.dtype == syn.DTYPE_FP8 else 0)
     q_bytes = wl.T * wl.H * slot_bytes
     w_bytes = wl.T * wl.H * 4
-    if wl.mode == syn.MODE_POSITIONS:
-        p = np.clip(np.asarray(inputs["positions"], np.int64) + 1, 0, wl.S)
-        k_slots = int(p.max()) if wl.shared_cache else int(p.sum())
+    if wl.mode != syn.MODE_CAUSAL:
+        p = np.clip(row_positions(wl, inputs) + 1, 0, wl.S)
+        shared = wl.shared_cache or wl.mode == syn.MODE_COMPRESSED
+        k_slots = int(p.max()) if shared else int(p.sum())
     else:
         k_slots = wl.T
     score_bytes = q_bytes + w_bytes + k_slots * slot_bytes + score_elems(wl) * 4
@@ -365,8 +375,8 @@ def run_e2e(args, wl, inputs, p, pairs, stream, device, dist):
 def oracle_sample_rows(wl, inputs, pair_budget: int, start: int = 0):
     """Query rows, taken round-robin from `start`, until the sample holds
     about `pair_budget` valid pairs (at least one row)."""
-    if wl.mode == syn.MODE_POSITIONS:
-        nv = np.clip(np.asarray(inputs["positions"], np.int64) + 1, 0, wl.S)
+    if wl.mode != syn.MODE_CAUSAL:
+        nv = np.clip(row_positions(wl, inputs) + 1, 0, wl.S)
     else:
         cu = wl.cu_seqlens().astype(np.int64)
         nv = np.empty(wl.T, np.int64)
@@ -445,10 +455,14 @@ def workload_config(wl, extra=None):
     c = {"workload": wl.name, "T": wl.T, "H": wl.H, "D": wl.D,
          "index_topk": wl.index_topk,
          "kv_dtype": "fp8_e4m3+e8m0/32" if wl.dtype == syn.DTYPE_FP8 else "bf16",
-         "mask": "positions" if wl.mode == syn.MODE_POSITIONS else "causal"}
+         "mask": {syn.MODE_POSITIONS: "positions", syn.MODE_CAUSAL: "causal",
+                  syn.MODE_COMPRESSED: "compressed"}[wl.mode]}
     if wl.mode == syn.MODE_POSITIONS:
         c.update(S=wl.S, positions=f"U[{wl.pos_lo},{wl.pos_hi})",
                  caches="shared" if wl.shared_cache else "one per token")
+    elif wl.mode == syn.MODE_COMPRESSED:
+        c.update(S=wl.S, compress_ratio=wl.compress_ratio, query_start=wl.query_start,
+                 caches="one pooled cache")
     else:
         c.update(seqlens=list(wl.seqlens))
     if extra:
@@ -493,7 +507,7 @@ def main(argv=None):
         return 0
     pk = peaks()
     value = r["pairs"] * world / (r["ms_step"] / 1e3)
-    tensor_bound = wl.mode == syn.MODE_CAUSAL or wl.shared_cache
+    tensor_bound = wl.mode != syn.MODE_POSITIONS or wl.shared_cache
     if tensor_bound:
         peak_t = pk["bf16"] * (2.0 if wl.dtype == syn.DTYPE_FP8 else 1.0)
         achieved = r["flops"] / (r["ms_score"] / 1e3) / 1e12

@@ -28,6 +28,14 @@
  *    Hadamard rotation because it is a no-op for q . k.
  *  - NeMo AutoModel optimized_kernels, sparse_attention_torch: a key index of
  *    -1 masks an entry.
+ *  - NeMo AutoModel optimized_kernels, dsv4_indexer_scores and
+ *    indexer_scores_torch: the DSV4 "C4" indexer scores queries against a
+ *    pooled (compressed) key cache, given compress_ratio and query_start.
+ *    The page gives the arguments, not the causal rule in pooled space; this
+ *    library reads it as: pooled slot j holds raw tokens [j*r, (j+1)*r) and
+ *    is valid for the query at absolute position query_start + t once all of
+ *    them have been seen, (j+1)*r <= query_start + t + 1. The softmax_scale
+ *    argument is a scalar factor of every score: fold it into w.
  *
  * Conventions common to every call:
  *  - Pointers are DEVICE pointers unless stated otherwise. The caller owns
@@ -75,10 +83,16 @@ typedef enum {
   DSA_MASK_POSITIONS = 0,  /* decode: token t reads cache t (or the one shared
                               cache); slot s valid iff s <= positions[t];
                               every score row has S entries                    */
-  DSA_MASK_CAUSAL = 1      /* packed prefill: sequences back to back as given
+  DSA_MASK_CAUSAL = 1,     /* packed prefill: sequences back to back as given
                               by cu_seqlens; token t of sequence i scores the
                               L_i keys of its own sequence; slot s valid iff
                               s <= t - cu_seqlens[i]                           */
+  DSA_MASK_COMPRESSED = 2  /* C4 indexer: every token scores the one pooled
+                              cache of S slots, each pooling compress_ratio
+                              raw tokens; token t sits at absolute position
+                              query_start + t and slot s is valid iff
+                              (s+1)*compress_ratio <= query_start + t + 1;
+                              every score row has S entries                    */
 } dsa_mask_t;
 
 /* The finite mask bound: the lowest finite bf16 value (bits 0xFF7F), exact
@@ -90,15 +104,21 @@ typedef struct {
   int32_t H;               /* indexer heads, 1 <= H <= 256                       */
   int32_t D;               /* head_dim; must be 128                              */
   int32_t index_topk;      /* k >= 1                                             */
-  int64_t S;               /* POSITIONS: slots per key cache, >= 1. CAUSAL: unused */
+  int64_t S;               /* POSITIONS: slots per key cache, >= 1.
+                              COMPRESSED: pooled slots, >= 1. CAUSAL: unused     */
   int64_t k_seq_stride;    /* POSITIONS: elements between consecutive tokens'
                               caches (a multiple of D, >= S*D), or 0 when every
-                              token reads one shared cache. CAUSAL: unused       */
+                              token reads one shared cache. COMPRESSED: must be
+                              0 (one pooled cache). CAUSAL: unused              */
   int32_t num_seqs;        /* CAUSAL: packed sequences, >= 1. POSITIONS: unused   */
   const int32_t *cu_seqlens; /* CAUSAL: device [num_seqs + 1], cu[0] = 0,
                               non-decreasing, cu[num_seqs] = T                  */
   dsa_kv_dtype_t dtype;
   dsa_mask_t mask;
+  int64_t query_start;     /* COMPRESSED: absolute position of token 0, >= 0.
+                              Otherwise unused                                  */
+  int32_t compress_ratio;  /* COMPRESSED: raw tokens per pooled slot, >= 1.
+                              Otherwise unused                                  */
 } dsa_indexer_desc_t;
 
 /*
@@ -107,13 +127,15 @@ typedef struct {
  *  q_scale  [T, H, D/32]   e8m0 bytes (FP8 only; NULL for BF16)
  *  w        [T, H]         fp32
  *  k        POSITIONS: cache of token t at element t*k_seq_stride, [S, D]
+ *           COMPRESSED: the pooled cache [S, D]
  *           CAUSAL:    [T, D], sequence i at rows cu[i] .. cu[i+1]-1
  *           bf16, or e4m3 bytes                                 (16-byte aligned)
  *  k_scale  same slots as k, [.., D/32] e8m0 bytes (FP8 only; NULL for BF16);
  *           POSITIONS cache t at byte t*(k_seq_stride/32)
- *  positions [T] int32 (POSITIONS only; NULL for CAUSAL). A negative position
- *           leaves the whole row masked.
- *  scores   POSITIONS: [T, S] fp32.
+ *  positions [T] int32 (POSITIONS only; ignored for CAUSAL; must be NULL
+ *           for COMPRESSED). A negative position leaves the whole row masked.
+ *  scores   POSITIONS, COMPRESSED: [T, S] fp32 (a COMPRESSED row that sees
+ *           no pooled slot is all mask bound, its top-k all -1).
  *           CAUSAL: sequence i's [L_i, L_i] block at float offset
  *           sum_{j<i} L_j^2; row t of it at + (t - cu[i]) * L_i.
  *  topk     [T, index_topk] int32, sequence-local 0-based slot indices in any
@@ -140,7 +162,8 @@ dsa_status_t dsa_indexer_score(const dsa_indexer_desc_t *desc,
                                dsa_stream_t stream);
 
 /* Top-k only, from score rows laid out as above (by this library or not);
- * validity comes from positions / cu_seqlens, never from the values.
+ * validity comes from positions / cu_seqlens / the compressed rule, never
+ * from the values.
  * Ties at the k-th score go to the lower slot. Asynchronous on `stream`. */
 dsa_status_t dsa_indexer_topk(const dsa_indexer_desc_t *desc,
                               const float *scores, const int32_t *positions,

@@ -27,6 +27,7 @@ DSA_KV_BF16 = 0
 DSA_KV_FP8_E4M3_E8M0_B32 = 1
 DSA_MASK_POSITIONS = 0
 DSA_MASK_CAUSAL = 1
+DSA_MASK_COMPRESSED = 2
 DSA_MASK_BOUND = float.fromhex("-0x1.FEp127")
 
 # Every symbol include/dsa_indexer.h declares.
@@ -40,7 +41,8 @@ class dsa_indexer_desc_t(ctypes.Structure):
                 ("D", ctypes.c_int32), ("index_topk", ctypes.c_int32),
                 ("S", ctypes.c_int64), ("k_seq_stride", ctypes.c_int64),
                 ("num_seqs", ctypes.c_int32), ("cu_seqlens", ctypes.c_void_p),
-                ("dtype", ctypes.c_int), ("mask", ctypes.c_int)]
+                ("dtype", ctypes.c_int), ("mask", ctypes.c_int),
+                ("query_start", ctypes.c_int64), ("compress_ratio", ctypes.c_int32)]
 
 
 class DsaError(RuntimeError):
@@ -81,11 +83,13 @@ def _ptr(x) -> int | None:
 
 
 def make_desc(T, H, index_topk, *, D=128, S=0, k_seq_stride=0, num_seqs=0,
-              cu_seqlens=None, dtype=DSA_KV_BF16, mask=DSA_MASK_POSITIONS):
+              cu_seqlens=None, dtype=DSA_KV_BF16, mask=DSA_MASK_POSITIONS,
+              query_start=0, compress_ratio=0):
     return dsa_indexer_desc_t(T=T, H=H, D=D, index_topk=index_topk, S=S,
                               k_seq_stride=k_seq_stride, num_seqs=num_seqs,
                               cu_seqlens=_ptr(cu_seqlens), dtype=dtype,
-                              mask=mask)
+                              mask=mask, query_start=query_start,
+                              compress_ratio=compress_ratio)
 
 
 def dsa_status_string(status: int) -> str:

@@ -98,7 +98,9 @@ dsa_status_t check_desc(const dsa_indexer_desc_t *d) {
   if (!d) return DSA_ERR_INVALID_ARG;
   if (d->T < 1 || d->H < 1 || d->index_topk < 1) return DSA_ERR_INVALID_ARG;
   if (d->dtype != DSA_KV_BF16 && d->dtype != DSA_KV_FP8_E4M3_E8M0_B32) return DSA_ERR_INVALID_ARG;
-  if (d->mask != DSA_MASK_POSITIONS && d->mask != DSA_MASK_CAUSAL) return DSA_ERR_INVALID_ARG;
+  if (d->mask != DSA_MASK_POSITIONS && d->mask != DSA_MASK_CAUSAL &&
+      d->mask != DSA_MASK_COMPRESSED)
+    return DSA_ERR_INVALID_ARG;
   if (d->D != 128) return DSA_ERR_UNSUPPORTED;
   if (d->H > 256) return DSA_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(d->T) * d->H > INT32_MAX - 256) return DSA_ERR_UNSUPPORTED;
@@ -108,6 +110,12 @@ dsa_status_t check_desc(const dsa_indexer_desc_t *d) {
     if (d->k_seq_stride != 0) {
       if (d->k_seq_stride < d->S * d->D || d->k_seq_stride % d->D != 0) return DSA_ERR_INVALID_ARG;
     }
+  } else if (d->mask == DSA_MASK_COMPRESSED) {
+    if (d->S < 1 || d->k_seq_stride != 0) return DSA_ERR_INVALID_ARG;
+    if (d->compress_ratio < 1 || d->query_start < 0) return DSA_ERR_INVALID_ARG;
+    if (d->S > INT32_MAX - 256) return DSA_ERR_UNSUPPORTED;
+    // the absolute positions must fit 64-bit arithmetic with room to spare
+    if (d->query_start > (INT64_MAX >> 2)) return DSA_ERR_UNSUPPORTED;
   } else {
     if (d->num_seqs < 1 || !d->cu_seqlens) return DSA_ERR_INVALID_ARG;
   }
@@ -304,7 +312,12 @@ dsa_status_t launch_score(const dsa_indexer_desc_t *d, const void *q, const uint
   p.shared_cache = d->k_seq_stride == 0;
   p.num_seqs = d->num_seqs;
   p.cu_seqlens = d->cu_seqlens;
-  p.positions = positions;
+  // COMPRESSED runs as POSITIONS over one shared cache, with no positions
+  // array: the kernels derive each row's last valid slot from the ratio.
+  const bool compressed = d->mask == DSA_MASK_COMPRESSED;
+  p.positions = compressed ? nullptr : positions;
+  p.query_start = compressed ? d->query_start : 0;
+  p.compress_ratio = compressed ? d->compress_ratio : 1;
   p.w = w;
   p.scores = scores;
   p.tq_sub = L.tq_sub;
@@ -337,7 +350,10 @@ dsa_status_t launch_topk(const dsa_indexer_desc_t *d, const float *scores,
   p.S = d->S;
   p.num_seqs = d->num_seqs;
   p.cu_seqlens = d->cu_seqlens;
-  p.positions = positions;
+  const bool compressed = d->mask == DSA_MASK_COMPRESSED;
+  p.positions = compressed ? nullptr : positions;
+  p.query_start = compressed ? d->query_start : 0;
+  p.compress_ratio = compressed ? d->compress_ratio : 1;
   p.scores = scores;
   p.topk = topk;
   p.k = d->index_topk;
@@ -377,6 +393,7 @@ dsa_status_t check_inputs(const dsa_indexer_desc_t *d, const void *q, const uint
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(w, 16) || !aligned(scores, 4))
     return DSA_ERR_INVALID_ARG;
   if (d->mask == DSA_MASK_POSITIONS && !positions) return DSA_ERR_INVALID_ARG;
+  if (d->mask == DSA_MASK_COMPRESSED && positions) return DSA_ERR_INVALID_ARG;
   if (d->dtype == DSA_KV_FP8_E4M3_E8M0_B32 && (!q_scale || !k_scale)) return DSA_ERR_INVALID_ARG;
   return DSA_OK;
 }
@@ -416,6 +433,7 @@ dsa_status_t dsa_indexer_topk(const dsa_indexer_desc_t *desc, const float *score
   if (st != DSA_OK) return st;
   if (!scores || !topk || !aligned(scores, 4) || !aligned(topk, 4)) return DSA_ERR_INVALID_ARG;
   if (desc->mask == DSA_MASK_POSITIONS && !positions) return DSA_ERR_INVALID_ARG;
+  if (desc->mask == DSA_MASK_COMPRESSED && positions) return DSA_ERR_INVALID_ARG;
   st = check_workspace(workspace, workspace_bytes);
   if (st != DSA_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

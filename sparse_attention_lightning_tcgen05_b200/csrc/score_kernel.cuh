@@ -36,6 +36,7 @@
 #include <cstdint>
 
 #include "sm100_ptx.cuh"
+#include "row_rule.cuh"
 
 namespace dsa {
 
@@ -52,7 +53,9 @@ struct ScoreParams {
   int shared_cache;          // POSITIONS: every token reads cache 0
   int num_seqs;              // CAUSAL
   const int *cu_seqlens;     // CAUSAL
-  const int *positions;      // POSITIONS
+  const int *positions;      // POSITIONS; NULL: the compressed rule
+  int64_t query_start;       // compressed rule: absolute position of token 0
+  int compress_ratio;        // compressed rule: raw tokens per pooled slot
   const float *w;            // [T, H]
   float *scores;
   int tq_sub;                // tokens per MMA sub-block (tq_sub*NSUB divides 128)
@@ -140,7 +143,8 @@ struct QBlk {
 };
 
 __device__ __forceinline__ int last_valid_pos(const ScoreParams &p, int t) {
-  const int pos = p.positions[t];     // global, or the CTA's shared copy
+  // positions: global, or the CTA's shared copy
+  const int64_t pos = row_position(p.positions, p.query_start, p.compress_ratio, t);
   const int64_t lv = pos < 0 ? -1 : (pos >= p.S ? p.S - 1 : pos);
   return static_cast<int>(lv);
 }
@@ -598,11 +602,20 @@ __global__ void __launch_bounds__((2 + kEPI + (kFP8 ? 1 : 0) + (kISS - 1)) * 32,
   grid_dep_wait();
   grid_dep_launch_dependents();
 
-  // Decode positions are read by every role many times: keep a copy here.
+  // Decode positions are read by every role many times: keep a copy here
+  // (with the compressed rule, the positions it gives, capped at S).
   int *spos = reinterpret_cast<int *>(smem + L.off_pos);
   const bool pos_staged = kMODE == kModePositions && p.T <= kPosCap;
-  if (pos_staged)
-    for (int i = threadIdx.x; i < p.T; i += blockDim.x) spos[i] = __ldg(p.positions + i);
+  if (pos_staged) {
+    if (p.positions) {
+      for (int i = threadIdx.x; i < p.T; i += blockDim.x) spos[i] = __ldg(p.positions + i);
+    } else {
+      for (int i = threadIdx.x; i < p.T; i += blockDim.x) {
+        const int64_t pos = row_position(nullptr, p.query_start, p.compress_ratio, i);
+        spos[i] = static_cast<int>(pos < p.S ? pos : p.S);
+      }
+    }
+  }
   __syncthreads();
   ScoreParams P = p;
   P.mode = kMODE;   // a constant from here on: the other mode's code folds away

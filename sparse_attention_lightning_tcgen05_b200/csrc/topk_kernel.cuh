@@ -24,6 +24,7 @@
 #include <cstdint>
 
 #include "sm100_ptx.cuh"
+#include "row_rule.cuh"
 
 namespace dsa {
 
@@ -36,7 +37,9 @@ struct TopkParams {
   int64_t S;                // POSITIONS row length
   int num_seqs;
   const int *cu_seqlens;
-  const int *positions;
+  const int *positions;     // POSITIONS; NULL: the compressed rule
+  int64_t query_start;      // compressed rule: absolute position of token 0
+  int compress_ratio;       // compressed rule: raw tokens per pooled slot
   const float *scores;
   int *topk;
   int k;
@@ -236,8 +239,8 @@ __global__ void __launch_bounds__(NT) topk_kernel(const TopkParams p) {
   int64_t nvalid;
   if (p.mode == kModePositions) {
     row = p.scores + static_cast<int64_t>(t) * p.S;
-    const int pos = __ldg(p.positions + t);
-    nvalid = pos < 0 ? 0 : (static_cast<int64_t>(pos) + 1 < p.S ? pos + 1 : p.S);
+    const int64_t pos = row_position(p.positions, p.query_start, p.compress_ratio, t);
+    nvalid = pos < 0 ? 0 : (pos + 1 < p.S ? pos + 1 : p.S);
   } else {
     if (tid == 0) {            // largest i with cu[i] <= t (cu non-decreasing)
       int lo = 0, hi = p.num_seqs - 1;

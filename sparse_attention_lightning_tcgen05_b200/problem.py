@@ -9,7 +9,7 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import (DSA_KV_BF16, DSA_MASK_CAUSAL, DSA_MASK_POSITIONS,
+from . import (DSA_KV_BF16, DSA_MASK_CAUSAL, DSA_MASK_COMPRESSED, DSA_MASK_POSITIONS,
                dsa_indexer_forward, dsa_indexer_get_error, dsa_indexer_score,
                dsa_indexer_topk, dsa_indexer_workspace_size, make_desc)
 
@@ -30,7 +30,8 @@ class DeviceProblem:
 
     def __init__(self, *, mode, T, H, index_topk, q, w, k, dtype=DSA_KV_BF16,
                  S=0, k_seq_stride=0, cu_seqlens=None, positions=None,
-                 q_scale=None, k_scale=None, device="cuda"):
+                 q_scale=None, k_scale=None, query_start=0, compress_ratio=0,
+                 device="cuda"):
         self.mode, self.T, self.H, self.k = mode, T, H, index_topk
         self.S, self.dtype = S, dtype
         self.q = _dev(q, device)
@@ -51,7 +52,8 @@ class DeviceProblem:
             n_scores = T * S
         self.desc = make_desc(T, H, index_topk, S=S, k_seq_stride=k_seq_stride,
                               num_seqs=self.num_seqs, cu_seqlens=self.cu_seqlens,
-                              dtype=dtype, mask=mode)
+                              dtype=dtype, mask=mode, query_start=query_start,
+                              compress_ratio=compress_ratio)
         self.scores = torch.empty(n_scores, dtype=torch.float32, device=device)
         self.topk = torch.empty((T, index_topk), dtype=torch.int32, device=device)
         self.ws_bytes = dsa_indexer_workspace_size(self.desc)
@@ -60,13 +62,15 @@ class DeviceProblem:
     @classmethod
     def from_workload(cls, wl, inputs, device="cuda"):
         """From a dsa_synth.Workload and its generated inputs."""
-        mode = DSA_MASK_CAUSAL if wl.mode == 1 else DSA_MASK_POSITIONS
+        mode = {0: DSA_MASK_POSITIONS, 1: DSA_MASK_CAUSAL,
+                2: DSA_MASK_COMPRESSED}[wl.mode]
         return cls(mode=mode, T=wl.T, H=wl.H, index_topk=wl.index_topk,
                    q=inputs["q"], w=inputs["w"], k=inputs["k"], dtype=wl.dtype,
                    S=wl.S, k_seq_stride=wl.k_seq_stride,
                    cu_seqlens=inputs.get("cu_seqlens"),
                    positions=inputs.get("positions"),
                    q_scale=inputs.get("q_scale"), k_scale=inputs.get("k_scale"),
+                   query_start=wl.query_start, compress_ratio=wl.compress_ratio,
                    device=device)
 
     def _stream(self, stream):

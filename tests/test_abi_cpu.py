@@ -61,6 +61,54 @@ def test_bad_descriptors(kw, code):
     assert e.value.status == code
 
 
+def compressed_desc(**kw):
+    d = dict(T=64, H=64, index_topk=16, S=300, k_seq_stride=0,
+             mask=dsa.DSA_MASK_COMPRESSED, compress_ratio=4, query_start=0)
+    d.update(kw)
+    return dsa.make_desc(**d)
+
+
+def test_compressed_descriptor_layout():
+    """The two compressed-mode fields sit after `mask`, 8-byte aligned, as the
+    C header declares them."""
+    import ctypes
+    f = dsa.dsa_indexer_desc_t
+    assert f.query_start.offset % 8 == 0 and f.query_start.offset > f.mask.offset
+    assert f.compress_ratio.offset == f.query_start.offset + 8
+    assert ctypes.sizeof(f) % 8 == 0
+    assert dsa.dsa_indexer_workspace_size(compressed_desc()) >= 256
+    assert dsa.dsa_indexer_workspace_size(compressed_desc(query_start=10**12,
+                                                          compress_ratio=1)) >= 256
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(compress_ratio=0), dsa.DSA_ERR_INVALID_ARG),
+    (dict(compress_ratio=-4), dsa.DSA_ERR_INVALID_ARG),
+    (dict(query_start=-1), dsa.DSA_ERR_INVALID_ARG),
+    (dict(S=0), dsa.DSA_ERR_INVALID_ARG),
+    (dict(k_seq_stride=300 * 128), dsa.DSA_ERR_INVALID_ARG),   # one pooled cache
+    (dict(query_start=1 << 62), dsa.DSA_ERR_UNSUPPORTED),
+    (dict(mask=3), dsa.DSA_ERR_INVALID_ARG),
+])
+def test_bad_compressed_descriptors(kw, code):
+    with pytest.raises(dsa.DsaError) as e:
+        dsa.dsa_indexer_workspace_size(compressed_desc(**kw))
+    assert e.value.status == code
+
+
+def test_compressed_rejects_a_positions_array():
+    d = compressed_desc()
+    fake = 1 << 20
+    for call in (lambda: dsa.dsa_indexer_forward(d, fake, None, fake, fake, None, fake,
+                                                 fake, fake, fake, 256),
+                 lambda: dsa.dsa_indexer_score(d, fake, None, fake, fake, None, fake,
+                                               fake, fake, 256),
+                 lambda: dsa.dsa_indexer_topk(d, fake, fake, fake, fake, 256)):
+        with pytest.raises(dsa.DsaError) as e:
+            call()
+        assert e.value.status == dsa.DSA_ERR_INVALID_ARG
+
+
 def test_bad_pointers_rejected_before_device_work():
     d = good_desc()
     fake = 1 << 20                     # never dereferenced: checks fail first

@@ -194,3 +194,56 @@ def test_long_decode_fp8_full_size_sampled(dsa):
 def test_fp8_decode_many_tokens(dsa):
     wl = fp8_decode_wl(T=70, H=64, S=1300, k=80, pos=(0, 1300), seed=41)
     run_and_check(dsa, wl, syn.generate(wl), tol=TOL_FP8)
+
+
+# ---- compressed (C4) keys: one pooled cache, validity from the ratio --------
+
+def c4_wl(T, H, S, k, r=4, qs=0, dtype=syn.DTYPE_BF16, seed=0):
+    return syn.Workload("c4", syn.MODE_COMPRESSED, T=T, H=H, D=128, index_topk=k,
+                        S=S, compress_ratio=r, query_start=qs, dtype=dtype,
+                        w_scale=1.0 / np.sqrt(H), seed=seed)
+
+
+@pytest.mark.parametrize("H", [4, 16, 64])
+def test_compressed_small(dsa, H):
+    """Rows that see no pooled slot, a few, and all of them; S ragged."""
+    wl = c4_wl(T=300, H=H, S=70, k=24, r=4, qs=0, seed=50 + H)
+    run_and_check(dsa, wl, syn.generate(wl))
+
+
+@pytest.mark.parametrize("H", [4, 64])
+def test_compressed_integer_inputs_bit_exact(dsa, H):
+    wl = c4_wl(T=200, H=H, S=140, k=32, r=3, qs=7, seed=51)
+    run_and_check(dsa, wl, syn.generate(wl, value_kind="int"), exact=True)
+
+
+def test_compressed_query_start_and_ratios(dsa):
+    """A late chunk (query_start past the pooled cache for some rows: those
+    rows are all valid) and a ratio of 1 (the causal rule on pooled keys)."""
+    for r, qs, T, S in ((4, 1000, 90, 300), (1, 37, 50, 120), (128, 0, 300, 5)):
+        wl = c4_wl(T=T, H=64, S=S, k=40, r=r, qs=qs, seed=52 + r)
+        run_and_check(dsa, wl, syn.generate(wl))
+
+
+def test_compressed_many_tokens_unstaged(dsa):
+    """More tokens than the score kernel stages in shared memory: every row
+    derives its last valid slot from the ratio on the fly."""
+    wl = c4_wl(T=2600, H=64, S=700, k=64, r=4, qs=5, seed=53)
+    rng = np.random.default_rng(14)
+    rows = sorted(set([0, 1, 2, 3, 4, 2047, 2048, 2599] +
+                      list(rng.integers(0, wl.T, 24))))
+    run_and_check(dsa, wl, syn.generate(wl), rows=rows)
+
+
+@pytest.mark.parametrize("H", [16, 64])
+def test_fp8_compressed(dsa, H):
+    wl = c4_wl(T=260, H=H, S=90, k=30, r=4, qs=3, dtype=syn.DTYPE_FP8, seed=54 + H)
+    run_and_check(dsa, wl, syn.generate(wl), tol=TOL_FP8)
+
+
+def test_c4_prefill_full_size_sampled(dsa):
+    wl = syn.WORKLOADS["c4_prefill"]
+    rng = np.random.default_rng(15)
+    rows = sorted(set([0, 2, 3, 4, 511, 4095, 4096, 8190, 8191] +
+                      list(rng.integers(0, wl.T, 12))))
+    run_and_check(dsa, wl, syn.generate(wl), rows=rows)

@@ -115,7 +115,9 @@ typedef struct {
                               non-decreasing, cu[num_seqs] = T                  */
   dsa_kv_dtype_t dtype;
   dsa_mask_t mask;
-  int64_t query_start;     /* COMPRESSED: absolute position of token 0, >= 0.
+  int64_t query_start;     /* COMPRESSED: absolute position of token 0, >= 0;
+                              query_start + T <= INT32_MAX (positions are 32-bit
+                              as in POSITIONS; DSA_ERR_UNSUPPORTED otherwise).
                               Otherwise unused                                  */
   int32_t compress_ratio;  /* COMPRESSED: raw tokens per pooled slot, >= 1.
                               Otherwise unused                                  */

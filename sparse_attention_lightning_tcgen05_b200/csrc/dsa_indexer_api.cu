@@ -114,8 +114,8 @@ dsa_status_t check_desc(const dsa_indexer_desc_t *d) {
     if (d->S < 1 || d->k_seq_stride != 0) return DSA_ERR_INVALID_ARG;
     if (d->compress_ratio < 1 || d->query_start < 0) return DSA_ERR_INVALID_ARG;
     if (d->S > INT32_MAX - 256) return DSA_ERR_UNSUPPORTED;
-    // the absolute positions must fit 64-bit arithmetic with room to spare
-    if (d->query_start > (INT64_MAX >> 2)) return DSA_ERR_UNSUPPORTED;
+    // absolute positions, like decode positions, are 32-bit
+    if (d->query_start > static_cast<int64_t>(INT32_MAX) - d->T) return DSA_ERR_UNSUPPORTED;
   } else {
     if (d->num_seqs < 1 || !d->cu_seqlens) return DSA_ERR_INVALID_ARG;
   }
@@ -125,6 +125,13 @@ dsa_status_t check_desc(const dsa_indexer_desc_t *d) {
     if (d->mask == DSA_MASK_POSITIONS && d->k_seq_stride % 512 != 0) return DSA_ERR_INVALID_ARG;
   }
   return DSA_OK;
+}
+
+// The compressed rule of a COMPRESSED descriptor (flag 0 otherwise).
+void set_compressed_rule(const dsa_indexer_desc_t *d, int &flag, dsa::CompressedRule &c) {
+  flag = d->mask == DSA_MASK_COMPRESSED;
+  c.base = flag ? static_cast<int32_t>(d->query_start + 1) : 1;
+  c.div = dsa::div_magic(flag ? static_cast<uint32_t>(d->compress_ratio) : 1u);
 }
 
 dsa_status_t check_workspace(const void *ws, size_t bytes) {
@@ -200,9 +207,29 @@ int pow2_floor(int x) {
 // per pipeline item. Prefill / a shared cache (H = 64): 8 tokens per query
 // block as two N = 256 sub-blocks. Any other H: the generic epilogue. Each
 // instance is compiled for one mask mode.
-constexpr int kPos = dsa::kModePositions, kCau = dsa::kModeCausal;
+constexpr int kPos = dsa::kModePositions, kCau = dsa::kModeCausal, kCmp = dsa::kModeCompressed;
+
+// COMPRESSED: the shared-cache instances, compiled with the compressed rule.
+ScoreLaunch choose_score_compressed(const dsa_indexer_desc_t *d) {
+  const int H = d->H;
+  if (d->dtype == DSA_KV_BF16) {
+    if (H == 64)
+      return {dsa::score_kernel<64, 2, 1, 2, 2, 1, 8, false, 1, kCmp>, 12, 2, 1, 2, 8, 1, 1, 4,
+              256, 256, false};
+    const int tq = pow2_floor(std::min(128, 256 / H));
+    return {dsa::score_kernel<0, 1, 1, 2, 4, 1, 4, false, 1, kCmp>, 13, 4, 1, 1, 4, 1, 1, tq,
+            round16(tq * H), 256, false};
+  }
+  if (H == 64)
+    return {dsa::score_kernel<64, 2, 1, 2, 4, 1, 8, true, 1, kCmp>, 14, 4, 1, 2, 8, 1, 1, 2, 128,
+            128, true};
+  const int tq = pow2_floor(std::min(128, 128 / H));
+  return {dsa::score_kernel<0, 1, 1, 2, 4, 1, 4, true, 1, kCmp>, 15, 4, 1, 1, 4, 1, 1, tq,
+          round16(tq * H), 128, true};
+}
 
 ScoreLaunch choose_score(const dsa_indexer_desc_t *d) {
+  if (d->mask == DSA_MASK_COMPRESSED) return choose_score_compressed(d);
   const bool causal = d->mask == DSA_MASK_CAUSAL;
   const bool per_token_cache = !causal && d->k_seq_stride != 0;
   const int H = d->H;
@@ -314,10 +341,8 @@ dsa_status_t launch_score(const dsa_indexer_desc_t *d, const void *q, const uint
   p.cu_seqlens = d->cu_seqlens;
   // COMPRESSED runs as POSITIONS over one shared cache, with no positions
   // array: the kernels derive each row's last valid slot from the ratio.
-  const bool compressed = d->mask == DSA_MASK_COMPRESSED;
-  p.positions = compressed ? nullptr : positions;
-  p.query_start = compressed ? d->query_start : 0;
-  p.compress_ratio = compressed ? d->compress_ratio : 1;
+  p.positions = positions;
+  set_compressed_rule(d, p.compressed, p.comp);
   p.w = w;
   p.scores = scores;
   p.tq_sub = L.tq_sub;
@@ -350,10 +375,8 @@ dsa_status_t launch_topk(const dsa_indexer_desc_t *d, const float *scores,
   p.S = d->S;
   p.num_seqs = d->num_seqs;
   p.cu_seqlens = d->cu_seqlens;
-  const bool compressed = d->mask == DSA_MASK_COMPRESSED;
-  p.positions = compressed ? nullptr : positions;
-  p.query_start = compressed ? d->query_start : 0;
-  p.compress_ratio = compressed ? d->compress_ratio : 1;
+  p.positions = positions;
+  set_compressed_rule(d, p.compressed, p.comp);
   p.scores = scores;
   p.topk = topk;
   p.k = d->index_topk;

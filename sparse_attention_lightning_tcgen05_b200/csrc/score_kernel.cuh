@@ -44,7 +44,9 @@ constexpr int kBlockM = 128;          // key slots per tile (MMA M)
 constexpr int kHeadDim = 128;         // D
 constexpr float kMaskBound = -0x1.FEp127f;   // lowest finite bf16
 
-enum : int { kModePositions = 0, kModeCausal = 1 };
+// COMPRESSED is POSITIONS over one shared cache with the last valid slot of
+// each row given by the compressed rule instead of a positions array.
+enum : int { kModePositions = 0, kModeCausal = 1, kModeCompressed = 2 };
 
 struct ScoreParams {
   int mode;
@@ -53,9 +55,9 @@ struct ScoreParams {
   int shared_cache;          // POSITIONS: every token reads cache 0
   int num_seqs;              // CAUSAL
   const int *cu_seqlens;     // CAUSAL
-  const int *positions;      // POSITIONS; NULL: the compressed rule
-  int64_t query_start;       // compressed rule: absolute position of token 0
-  int compress_ratio;        // compressed rule: raw tokens per pooled slot
+  const int *positions;      // POSITIONS
+  int compressed;            // POSITIONS geometry, rows end by the compressed rule
+  CompressedRule comp;
   const float *w;            // [T, H]
   float *scores;
   int tq_sub;                // tokens per MMA sub-block (tq_sub*NSUB divides 128)
@@ -144,7 +146,7 @@ struct QBlk {
 
 __device__ __forceinline__ int last_valid_pos(const ScoreParams &p, int t) {
   // positions: global, or the CTA's shared copy
-  const int64_t pos = row_position(p.positions, p.query_start, p.compress_ratio, t);
+  const int64_t pos = p.compressed ? compressed_last_slot(p.comp, t) : p.positions[t];
   const int64_t lv = pos < 0 ? -1 : (pos >= p.S ? p.S - 1 : pos);
   return static_cast<int>(lv);
 }
@@ -523,8 +525,8 @@ __device__ __forceinline__ void sf_reorder_atom(const uint32_t *rows, int nrows,
 // kFP8: e4m3 + e8m0/32 inputs through the block-scaled MMA.
 // kISS: MMA-issuing warps (1 or 2). With 2, items alternate between them so
 //     that one warp's waits and commits overlap the other's MMAs.
-// kMODE: kModePositions or kModeCausal, fixed at compile time so that each
-//     instance carries only its own schedule code.
+// kMODE: kModePositions, kModeCausal or kModeCompressed, fixed at compile
+//     time so that each instance carries only its own schedule and row rule.
 //
 // Warps: 0 TMA producer, 1 MMA issuer (+ TMEM owner), 2 .. 1+kEPI epilogue,
 // then (fp8) the scale-factor warp, then (kISS == 2) the second issuer.
@@ -602,23 +604,16 @@ __global__ void __launch_bounds__((2 + kEPI + (kFP8 ? 1 : 0) + (kISS - 1)) * 32,
   grid_dep_wait();
   grid_dep_launch_dependents();
 
-  // Decode positions are read by every role many times: keep a copy here
-  // (with the compressed rule, the positions it gives, capped at S).
+  // Decode positions are read by every role many times: keep a copy here.
   int *spos = reinterpret_cast<int *>(smem + L.off_pos);
   const bool pos_staged = kMODE == kModePositions && p.T <= kPosCap;
-  if (pos_staged) {
-    if (p.positions) {
-      for (int i = threadIdx.x; i < p.T; i += blockDim.x) spos[i] = __ldg(p.positions + i);
-    } else {
-      for (int i = threadIdx.x; i < p.T; i += blockDim.x) {
-        const int64_t pos = row_position(nullptr, p.query_start, p.compress_ratio, i);
-        spos[i] = static_cast<int>(pos < p.S ? pos : p.S);
-      }
-    }
-  }
+  if (pos_staged)
+    for (int i = threadIdx.x; i < p.T; i += blockDim.x) spos[i] = __ldg(p.positions + i);
   __syncthreads();
   ScoreParams P = p;
-  P.mode = kMODE;   // a constant from here on: the other mode's code folds away
+  // constants from here on: the other modes' code folds away
+  P.mode = kMODE == kModeCompressed ? static_cast<int>(kModePositions) : kMODE;
+  P.compressed = kMODE == kModeCompressed;
   if (pos_staged) P.positions = spos;
   if (warp == 0) {
     CtaRange R;

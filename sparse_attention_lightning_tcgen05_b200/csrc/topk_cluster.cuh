@@ -206,7 +206,7 @@ __global__ void __launch_bounds__(NT) topk_cluster_kernel(const TopkParams p) {
   grid_dep_launch_dependents();
 
   const float *row = p.scores + static_cast<int64_t>(t) * p.S;
-  const int64_t pos = row_position(p.positions, p.query_start, p.compress_ratio, t);
+  const int64_t pos = p.compressed ? compressed_last_slot(p.comp, t) : __ldg(p.positions + t);
   const int64_t nvalid = pos < 0 ? 0 : (pos + 1 < p.S ? pos + 1 : p.S);
   int *out = p.topk + static_cast<int64_t>(t) * p.k;
   const uint32_t k = static_cast<uint32_t>(p.k);

@@ -37,9 +37,9 @@ struct TopkParams {
   int64_t S;                // POSITIONS row length
   int num_seqs;
   const int *cu_seqlens;
-  const int *positions;     // POSITIONS; NULL: the compressed rule
-  int64_t query_start;      // compressed rule: absolute position of token 0
-  int compress_ratio;       // compressed rule: raw tokens per pooled slot
+  const int *positions;     // POSITIONS
+  int compressed;           // POSITIONS rows that end by the compressed rule
+  CompressedRule comp;
   const float *scores;
   int *topk;
   int k;
@@ -239,7 +239,7 @@ __global__ void __launch_bounds__(NT) topk_kernel(const TopkParams p) {
   int64_t nvalid;
   if (p.mode == kModePositions) {
     row = p.scores + static_cast<int64_t>(t) * p.S;
-    const int64_t pos = row_position(p.positions, p.query_start, p.compress_ratio, t);
+    const int64_t pos = p.compressed ? compressed_last_slot(p.comp, t) : __ldg(p.positions + t);
     nvalid = pos < 0 ? 0 : (pos + 1 < p.S ? pos + 1 : p.S);
   } else {
     if (tid == 0) {            // largest i with cu[i] <= t (cu non-decreasing)

@@ -77,8 +77,8 @@ def test_compressed_descriptor_layout():
     assert f.compress_ratio.offset == f.query_start.offset + 8
     assert ctypes.sizeof(f) % 8 == 0
     assert dsa.dsa_indexer_workspace_size(compressed_desc()) >= 256
-    assert dsa.dsa_indexer_workspace_size(compressed_desc(query_start=10**12,
-                                                          compress_ratio=1)) >= 256
+    assert dsa.dsa_indexer_workspace_size(
+        compressed_desc(query_start=2**31 - 1 - 64, compress_ratio=1)) >= 256
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -88,6 +88,7 @@ def test_compressed_descriptor_layout():
     (dict(S=0), dsa.DSA_ERR_INVALID_ARG),
     (dict(k_seq_stride=300 * 128), dsa.DSA_ERR_INVALID_ARG),   # one pooled cache
     (dict(query_start=1 << 62), dsa.DSA_ERR_UNSUPPORTED),
+    (dict(query_start=2**31 - 64), dsa.DSA_ERR_UNSUPPORTED),   # 32-bit positions
     (dict(mask=3), dsa.DSA_ERR_INVALID_ARG),
 ])
 def test_bad_compressed_descriptors(kw, code):
@@ -159,3 +160,48 @@ def test_noalloc_rejects_bad_arguments_on_the_host():
         dsa.dsa_indexer_forward_noalloc(good_desc(D=64), fake, None, fake, fake, None,
                                         fake, fake, fake)
     assert e.value.status == dsa.DSA_ERR_UNSUPPORTED
+
+
+ROW_RULE = os.path.join(os.path.dirname(dsa.LIB_PATH), "csrc", "row_rule.cuh")
+_DIV_CHECK = r"""
+#include <cstdio>
+#include <cstdlib>
+#include "row_rule.cuh"
+// Every divisor in a list against plain integer division, on numerators
+// spread over [0, 2^31) plus the ones next to multiples of the divisor.
+int main() {
+  const uint32_t ds[] = {1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11, 12, 13, 16, 17, 31, 32, 33, 64,
+                         100, 127, 128, 129, 255, 256, 1000, 4095, 4096, 65535, 65536,
+                         65537, 1000003, 16777216, 16777217, 1073741823, 1073741824,
+                         1073741825, 2147483646, 2147483647};
+  unsigned long long bad = 0, n_checked = 0;
+  for (uint32_t d : ds) {
+    const dsa::DivMagic g = dsa::div_magic(d);
+    auto check = [&](uint64_t n) {
+      if (n >= (1ull << 31)) return;
+      ++n_checked;
+      if (dsa::div_by(static_cast<uint32_t>(n), g) != n / d) ++bad;
+    };
+    for (uint64_t n = 0; n < 4096; ++n) check(n);
+    for (uint64_t n = 0; n < (1ull << 31); n += 65521 + d % 7) check(n);
+    for (uint64_t q = 1; q < 4096; ++q) { check(q * d - 1); check(q * d); check(q * d + 1); }
+    for (uint64_t n = (1ull << 31) - 4096; n < (1ull << 31); ++n) check(n);
+  }
+  std::printf("%llu %llu\n", bad, n_checked);
+  return bad != 0;
+}
+"""
+
+
+def test_invariant_division_of_the_compressed_rule(tmp_path):
+    """The kernels' multiply-and-shift division by compress_ratio equals
+    integer division for 31-bit numerators (host build of the same header)."""
+    import subprocess
+    src = tmp_path / "div_check.cpp"
+    src.write_text(_DIV_CHECK)
+    exe = tmp_path / "div_check"
+    subprocess.run(["g++", "-O2", "-std=c++17", "-I", os.path.dirname(ROW_RULE), str(src),
+                    "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    bad, n = map(int, out.stdout.split())
+    assert out.returncode == 0 and bad == 0 and n > 10**6

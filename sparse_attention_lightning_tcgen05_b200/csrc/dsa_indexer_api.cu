@@ -350,6 +350,11 @@ dsa_status_t launch_score(const dsa_indexer_desc_t *d, const void *q, const uint
   p.err = &ws->err;
   p.err_info = &ws->err_info;
   p.wait_limit_ns = kWaitLimitNs;
+  // With one query buffer the next block's query cannot load while the
+  // current block's MMAs run: a block start costs about 3/4 of a key tile
+  // (measured on an 8192-token prefill), so the split between CTAs counts
+  // it. Double-buffered queries hide it.
+  p.blk_w = L.qbuf == 1 ? 6 : 0;
 
   int grid = dev->num_sms;
   if (!causal) {

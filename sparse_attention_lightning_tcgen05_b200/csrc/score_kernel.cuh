@@ -19,7 +19,9 @@
 // one key cache. An "active item" is (query block, key tile) with the tile
 // holding at least one valid slot of the block; a "fill item" is a tile of the
 // block's score rows where every slot is masked. Both lists are split into
-// equal contiguous ranges, one per CTA (no atomics, balanced to one tile).
+// contiguous ranges, one per CTA (no atomics), by cost: a query block's own
+// cost (its query load and pipeline refill; the fixed time of its fill
+// stores) counts beside its tiles.
 // Per active item the MMA issues one accumulator per sub-block; accumulators
 // rotate through NACC TMEM buffers so the epilogue of one overlaps the MMA of
 // the next. Fill items are never loaded: the epilogue writes the mask bound,
@@ -58,6 +60,7 @@ struct ScoreParams {
   const int *positions;      // POSITIONS
   int compressed;            // POSITIONS geometry, rows end by the compressed rule
   CompressedRule comp;
+  int blk_w;                 // schedule weight of a query block (a key tile weighs 8)
   const float *w;            // [T, H]
   float *scores;
   int tq_sub;                // tokens per MMA sub-block (tq_sub*NSUB divides 128)
@@ -172,7 +175,21 @@ __device__ __forceinline__ void make_qb_positions(const ScoreParams &p, int tqt,
   q.seqoff = 0;
   q.lv0 = 0;
   int mx = -1;
-  for (int i = 0; i < q.ntok; ++i) mx = max(mx, last_valid_pos(p, q.t0 + i));
+  if (p.compressed) {
+    // the compressed rule never decreases along the tokens
+    if (q.ntok > 0) mx = last_valid_pos(p, q.t0 + q.ntok - 1);
+  } else {
+    int m1 = -1, m2 = -1, m3 = -1;      // four independent chains
+    int i = 0;
+    for (; i + 4 <= q.ntok; i += 4) {
+      mx = max(mx, last_valid_pos(p, q.t0 + i));
+      m1 = max(m1, last_valid_pos(p, q.t0 + i + 1));
+      m2 = max(m2, last_valid_pos(p, q.t0 + i + 2));
+      m3 = max(m3, last_valid_pos(p, q.t0 + i + 3));
+    }
+    for (; i < q.ntok; ++i) mx = max(mx, last_valid_pos(p, q.t0 + i));
+    mx = max(max(mx, m1), max(m2, m3));
+  }
   q.ntr = static_cast<int>((p.S + kBlockM - 1) / kBlockM);
   q.act = mx < 0 ? 0 : mx / kBlockM + 1;
 }
@@ -236,79 +253,144 @@ struct CtaRange {
   int64_t a_seqoff, f_seqoff;
 };
 
-// POSITIONS: this CTA's share of both lists in two warp-wide passes over the
-// query blocks. Pass 1 sums the active and fill tiles; each lane 0..3 then
-// forms one bound (A*c/G, A*(c+1)/G, F*c/G, F*(c+1)/G) so that the four
-// divisions overlap. Pass 2 scans the blocks again, 32 at a time, and finds
-// the blocks holding items a0 and f0. A chunk of 32 blocks holds fewer than
-// 2^29 tiles (a row has at most 2^24), so the scans inside a chunk are
-// 32-bit; only the running bases are 64-bit. Full warp.
+// Both lists are split between CTAs by cost, not by count. An active tile
+// weighs kTileW and every query block with an active tile adds blk_w (its
+// query load and the pipeline refill at its start); a fill tile weighs
+// kFillTileW and every block with a fill tile adds kFillBlkW (the epilogue's
+// walk to the block and the fixed time of its row stores). With a list's
+// weights laid end to end, tile j of a block whose weights start at P sits at
+// P + (block weight) + (tile weight)*j, and CTA c of G takes the tiles
+// sitting in [Wt*c/G, Wt*(c+1)/G) (Wt: the list's total), so a CTA whose
+// share crosses many short blocks takes fewer tiles.
+constexpr int kTileW = 8;
+constexpr int kFillTileW = 1;
+constexpr int kFillBlkW = 10;
+
+// Of the n tiles of a block whose weights start at P, the number sitting
+// before weight w.
+__device__ __forceinline__ int tiles_before(int64_t w, int64_t P, int64_t blk_w, int tile_w,
+                                            int n) {
+  const int64_t num = w - P - blk_w;
+  if (num <= 0) return 0;
+  const int64_t k = (num + tile_w - 1) / tile_w;
+  return k < n ? static_cast<int>(k) : n;
+}
+
+// Inclusive warp scan.
+__device__ __forceinline__ int64_t warp_incl_scan(int64_t v, int lane) {
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int64_t n = __shfl_up_sync(0xffffffffu, v, off);
+    if (lane >= off) v += n;
+  }
+  return v;
+}
+
+// POSITIONS: this CTA's share of both lists, by one warp in one pass over
+// the query blocks. Lane l owns a contiguous run of blocks and totals both
+// lists' tiles and blocks over it; one warp scan places the runs and gives
+// the totals; lanes 0..3 form the four bounds (w0, w1 of the active list,
+// v0, v1 of the fill list) so that their divisions overlap; the lane whose
+// run holds the first tile at or after a bound walks its run again to find
+// it, and broadcasts it. Full warp.
 __device__ __forceinline__ void cta_range_positions(const ScoreParams &p, int tqt, CtaRange &R) {
   const int lane = threadIdx.x & 31;
   const int nqb = pos_num_blocks(p, tqt);
-  int64_t a = 0, f = 0;
-  for (int b = lane; b < nqb; b += 32) {
+  const int64_t bw = p.blk_w;
+  const int per = (nqb + 31) / 32;
+  const int lo = min(nqb, lane * per), hi = min(nqb, lo + per);
+  int64_t sa = 0, sc = 0, sf = 0, sfb = 0;
+  for (int b = lo; b < hi; ++b) {
     QBlk q;
     make_qb_positions(p, tqt, b, q);
-    a += q.act;
-    f += q.ntr - q.act;
+    sa += q.act;
+    sc += q.act > 0;
+    sf += q.ntr - q.act;
+    sfb += q.ntr > q.act;
   }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    a += __shfl_xor_sync(0xffffffffu, a, off);
-    f += __shfl_xor_sync(0xffffffffu, f, off);
-  }
+  const int64_t ia = warp_incl_scan(sa, lane), ic = warp_incl_scan(sc, lane);
+  const int64_t jf = warp_incl_scan(sf, lane), jfb = warp_incl_scan(sfb, lane);
+  const int64_t A = __shfl_sync(0xffffffffu, ia, 31), NB = __shfl_sync(0xffffffffu, ic, 31);
+  const int64_t F = __shfl_sync(0xffffffffu, jf, 31), NFB = __shfl_sync(0xffffffffu, jfb, 31);
+  const int64_t wa = kTileW * A + bw * NB;
+  const int64_t wf = kFillTileW * F + kFillBlkW * NFB;
   int64_t bound = 0;
-  if (lane < 4) bound = (lane < 2 ? a : f) * (blockIdx.x + (lane & 1)) / gridDim.x;
-  const int64_t a0 = __shfl_sync(0xffffffffu, bound, 0);
-  const int64_t a1 = __shfl_sync(0xffffffffu, bound, 1);
-  const int64_t f0 = __shfl_sync(0xffffffffu, bound, 2);
-  const int64_t f1 = __shfl_sync(0xffffffffu, bound, 3);
-  R.a_count = a1 - a0;
-  R.f_count = f1 - f0;
-  R.a_seq = R.f_seq = 0;
-  R.a_b = R.f_b = nqb;
-  R.a_j = R.f_j = 0;
-  R.a_seqoff = R.f_seqoff = 0;
-  bool need_a = R.a_count > 0, need_f = R.f_count > 0;
-  int64_t abase = 0, fbase = 0;
-  for (int c0 = 0; c0 < nqb && (need_a || need_f); c0 += 32) {
-    const int b = c0 + lane;
-    int act = 0, fil = 0;
-    if (b < nqb) {
-      QBlk q;
-      make_qb_positions(p, tqt, b, q);
-      act = q.act;
-      fil = q.ntr - q.act;
-    }
-    int ia = act, jf = fil;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int na = __shfl_up_sync(0xffffffffu, ia, off);
-      const int nf = __shfl_up_sync(0xffffffffu, jf, off);
-      if (lane >= off) {
-        ia += na;
-        jf += nf;
+  if (lane < 4) bound = (lane < 2 ? wa : wf) * (blockIdx.x + (lane & 1)) / gridDim.x;
+  const int64_t w0 = __shfl_sync(0xffffffffu, bound, 0);
+  const int64_t w1 = __shfl_sync(0xffffffffu, bound, 1);
+  const int64_t v0 = __shfl_sync(0xffffffffu, bound, 2);
+  const int64_t v1 = __shfl_sync(0xffffffffu, bound, 3);
+  // where this lane's weights start and where its last tile sits
+  const int64_t Pa = kTileW * (ia - sa) + bw * (ic - sc);
+  const int64_t Pf = kFillTileW * (jf - sf) + kFillBlkW * (jfb - sfb);
+  const int64_t La = kTileW * ia + bw * ic - kTileW;
+  const int64_t Lf = kFillTileW * jf + kFillBlkW * jfb - kFillTileW;
+  const int l_w0 = __ffs(__ballot_sync(0xffffffffu, w0 < wa && sa > 0 && La >= w0)) - 1;
+  const int l_w1 = __ffs(__ballot_sync(0xffffffffu, w1 < wa && sa > 0 && La >= w1)) - 1;
+  const int l_v0 = __ffs(__ballot_sync(0xffffffffu, v0 < wf && sf > 0 && Lf >= v0)) - 1;
+  const int l_v1 = __ffs(__ballot_sync(0xffffffffu, v1 < wf && sf > 0 && Lf >= v1)) - 1;
+  // The owners walk their runs again. g*, h*: list index of the tile found,
+  // or the list's length (no tile at or after the bound).
+  int a_b = nqb, a_j = 0, f_b = nqb, f_j = 0;
+  int64_t g0 = A, g1 = A, h0 = F, h1 = F;
+  bool n_w0 = lane == l_w0, n_w1 = lane == l_w1, n_v0 = lane == l_v0, n_v1 = lane == l_v1;
+  int64_t P = Pa, Q = Pf, ga = ia - sa, gf = jf - sf;
+  for (int b = lo; b < hi && (n_w0 || n_w1 || n_v0 || n_v1); ++b) {
+    QBlk q;
+    make_qb_positions(p, tqt, b, q);
+    const int act = q.act, fil = q.ntr - q.act;
+    if (act > 0) {
+      const int64_t last = P + bw + static_cast<int64_t>(kTileW) * (act - 1);
+      if (n_w0 && last >= w0) {
+        a_b = b;
+        a_j = tiles_before(w0, P, bw, kTileW, act);
+        g0 = ga + a_j;
+        n_w0 = false;
       }
+      if (n_w1 && last >= w1) {
+        g1 = ga + tiles_before(w1, P, bw, kTileW, act);
+        n_w1 = false;
+      }
+      P += bw + static_cast<int64_t>(kTileW) * act;
+      ga += act;
     }
-    const unsigned hit_a = __ballot_sync(0xffffffffu, need_a && abase + ia > a0);
-    const unsigned hit_f = __ballot_sync(0xffffffffu, need_f && fbase + jf > f0);
-    if (hit_a) {
-      const int l = __ffs(hit_a) - 1;
-      R.a_b = c0 + l;
-      R.a_j = static_cast<int>(a0 - abase - __shfl_sync(0xffffffffu, ia - act, l));
-      need_a = false;
+    if (fil > 0) {
+      const int64_t last = Q + kFillBlkW + static_cast<int64_t>(kFillTileW) * (fil - 1);
+      if (n_v0 && last >= v0) {
+        const int j = tiles_before(v0, Q, kFillBlkW, kFillTileW, fil);
+        f_b = b;
+        f_j = act + j;          // fill tiles follow the row's active ones
+        h0 = gf + j;
+        n_v0 = false;
+      }
+      if (n_v1 && last >= v1) {
+        h1 = gf + tiles_before(v1, Q, kFillBlkW, kFillTileW, fil);
+        n_v1 = false;
+      }
+      Q += kFillBlkW + static_cast<int64_t>(kFillTileW) * fil;
+      gf += fil;
     }
-    if (hit_f) {
-      const int l = __ffs(hit_f) - 1;
-      R.f_b = c0 + l;
-      R.f_j = static_cast<int>(f0 - fbase - __shfl_sync(0xffffffffu, jf - fil, l)) +
-              __shfl_sync(0xffffffffu, act, l);
-      need_f = false;
-    }
-    abase += __shfl_sync(0xffffffffu, ia, 31);
-    fbase += __shfl_sync(0xffffffffu, jf, 31);
   }
+  R.a_seq = R.f_seq = 0;
+  R.a_seqoff = R.f_seqoff = 0;
+  R.a_b = nqb;
+  R.a_j = 0;
+  R.f_b = nqb;
+  R.f_j = 0;
+  if (l_w0 >= 0) {
+    R.a_b = __shfl_sync(0xffffffffu, a_b, l_w0);
+    R.a_j = __shfl_sync(0xffffffffu, a_j, l_w0);
+    g0 = __shfl_sync(0xffffffffu, g0, l_w0);
+  }
+  if (l_w1 >= 0) g1 = __shfl_sync(0xffffffffu, g1, l_w1);
+  if (l_v0 >= 0) {
+    R.f_b = __shfl_sync(0xffffffffu, f_b, l_v0);
+    R.f_j = __shfl_sync(0xffffffffu, f_j, l_v0);
+    h0 = __shfl_sync(0xffffffffu, h0, l_v0);
+  }
+  if (l_v1 >= 0) h1 = __shfl_sync(0xffffffffu, h1, l_v1);
+  R.a_count = g1 - g0;
+  R.f_count = h1 - h0;
 }
 
 // CAUSAL: active or fill items before block B of a sequence.
@@ -317,47 +399,75 @@ __device__ __forceinline__ int64_t causal_before(int64_t B, int r, int ntr, bool
   return fill ? B * ntr - a : a;
 }
 
-// CAUSAL: locate item idx of the active or fill list (one thread).
-__device__ __forceinline__ void locate_causal(const ScoreParams &p, int tqt, int64_t idx, bool fill,
-                              int &seq_out, int &b_out, int &j_out, int64_t &seqoff_out) {
+// CAUSAL: weight of blocks [0, B) of a sequence in the active list (every
+// block holds an active tile) or in the fill list (block b holds ntr - b/r - 1
+// fill tiles: those below b < r*(ntr-1) hold one).
+__device__ __forceinline__ int64_t causal_weight_before(int64_t B, int r, int ntr, int64_t bw,
+                                                        bool fill) {
+  const int64_t act = causal_active_before(B, r);
+  if (!fill) return kTileW * act + bw * B;
+  const int64_t with_fill = static_cast<int64_t>(r) * (ntr - 1);
+  return kFillTileW * (B * ntr - act) + kFillBlkW * (B < with_fill ? B : with_fill);
+}
+
+// CAUSAL: the first tile of the active or fill list sitting at or after
+// weight w -- its sequence, block, tile in the score row and the sequence's
+// score offset -- and its index in the list (the list's length when there is
+// none). One thread.
+__device__ __forceinline__ int64_t locate_causal_weight(const ScoreParams &p, int tqt, int64_t w,
+                                                        bool fill, int &seq_out, int &b_out,
+                                                        int &j_out, int64_t &seqoff_out) {
   const int r = kBlockM / tqt;
-  int64_t off = 0;
+  const int64_t bw = fill ? kFillBlkW : p.blk_w;
+  const int tw = fill ? kFillTileW : kTileW;
+  int64_t off = 0, gbase = 0;
   for (int s = 0; s < p.num_seqs; ++s) {
     const int L = __ldg(p.cu_seqlens + s + 1) - __ldg(p.cu_seqlens + s);
     if (L <= 0) continue;
     const int nqb = (L + tqt - 1) / tqt, ntr = (L + kBlockM - 1) / kBlockM;
-    const int64_t tot = causal_before(nqb, r, ntr, fill);
-    if (idx < tot) {
-      int lo = 0, hi = nqb - 1;                 // last block whose prefix <= idx
+    const int64_t tot = causal_weight_before(nqb, r, ntr, bw, fill);
+    if (w <= tot - tw) {              // the sequence's last tile sits at tot - tw
+      int lo = 0, hi = nqb - 1;       // first block whose last tile sits at or after w
       while (lo < hi) {
-        const int mid = (lo + hi + 1) / 2;
-        if (causal_before(mid, r, ntr, fill) <= idx) lo = mid; else hi = mid - 1;
+        const int mid = (lo + hi) / 2;
+        if (causal_weight_before(mid + 1, r, ntr, bw, fill) - tw >= w) hi = mid; else lo = mid + 1;
       }
+      const int act = lo / r + 1, n = fill ? ntr - act : act;
+      const int j = tiles_before(w, causal_weight_before(lo, r, ntr, bw, fill), bw, tw, n);
       seq_out = s;
       b_out = lo;
-      j_out = static_cast<int>(idx - causal_before(lo, r, ntr, fill)) + (fill ? lo / r + 1 : 0);
+      j_out = fill ? act + j : j;
       seqoff_out = off;
-      return;
+      return gbase + causal_before(lo, r, ntr, fill) + j;
     }
-    idx -= tot;
+    w -= tot;
+    gbase += causal_before(nqb, r, ntr, fill);
     off += static_cast<int64_t>(L) * L;
   }
   seq_out = p.num_seqs;
   b_out = 0;
   j_out = 0;
   seqoff_out = off;
+  return gbase;
 }
 
-__device__ __forceinline__ void count_causal(const ScoreParams &p, int tqt, int64_t &A, int64_t &F) {
+// CAUSAL: active tiles A, fill tiles F, query blocks NB and blocks holding a
+// fill tile NFB of the batch.
+__device__ __forceinline__ void count_causal(const ScoreParams &p, int tqt, int64_t &A, int64_t &F,
+                                             int64_t &NB, int64_t &NFB) {
   const int r = kBlockM / tqt;
   A = 0;
   F = 0;
+  NB = 0;
+  NFB = 0;
   for (int s = 0; s < p.num_seqs; ++s) {
     const int L = __ldg(p.cu_seqlens + s + 1) - __ldg(p.cu_seqlens + s);
     if (L <= 0) continue;
     const int nqb = (L + tqt - 1) / tqt, ntr = (L + kBlockM - 1) / kBlockM;
     A += causal_before(nqb, r, ntr, false);
     F += causal_before(nqb, r, ntr, true);
+    NB += nqb;
+    NFB += nqb < r * (ntr - 1) ? nqb : r * (ntr - 1);
   }
 }
 
@@ -369,18 +479,30 @@ __device__ __forceinline__ void cta_range(const ScoreParams &p, int tqt, CtaRang
     return;
   }
   const int64_t G = gridDim.x, c = blockIdx.x;
-  int64_t A = 0, F = 0;
-  count_causal(p, tqt, A, F);
-  const int64_t a0 = A * c / G, a1 = A * (c + 1) / G;
-  const int64_t f0 = F * c / G, f1 = F * (c + 1) / G;
-  R.a_count = a1 - a0;
-  R.f_count = f1 - f0;
+  int64_t A = 0, F = 0, NB = 0, NFB = 0;
+  count_causal(p, tqt, A, F, NB, NFB);
+  const int64_t wa = kTileW * A + p.blk_w * NB;
+  const int64_t wf = kFillTileW * F + kFillBlkW * NFB;
+  const int64_t w0 = wa * c / G, w1 = wa * (c + 1) / G;
+  const int64_t v0 = wf * c / G, v1 = wf * (c + 1) / G;
   R.a_seq = R.f_seq = 0;
   R.a_b = R.f_b = 0;
   R.a_j = R.f_j = 0;
   R.a_seqoff = R.f_seqoff = 0;
-  if (R.a_count > 0) locate_causal(p, tqt, a0, false, R.a_seq, R.a_b, R.a_j, R.a_seqoff);
-  if (R.f_count > 0) locate_causal(p, tqt, f0, true, R.f_seq, R.f_b, R.f_j, R.f_seqoff);
+  R.a_count = 0;
+  R.f_count = 0;
+  int s1, b1, j1;
+  int64_t off1;
+  if (w0 < wa) {
+    const int64_t g0 =
+        locate_causal_weight(p, tqt, w0, false, R.a_seq, R.a_b, R.a_j, R.a_seqoff);
+    R.a_count = locate_causal_weight(p, tqt, w1, false, s1, b1, j1, off1) - g0;
+  }
+  if (v0 < wf) {
+    const int64_t h0 =
+        locate_causal_weight(p, tqt, v0, true, R.f_seq, R.f_b, R.f_j, R.f_seqoff);
+    R.f_count = locate_causal_weight(p, tqt, v1, true, s1, b1, j1, off1) - h0;
+  }
 }
 
 __device__ __forceinline__ void make_qb(const ScoreParams &p, int tqt, int seq, int b,
@@ -867,19 +989,27 @@ __global__ void __launch_bounds__((2 + kEPI + (kFP8 ? 1 : 0) + (kISS - 1)) * 32,
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
     // Fully masked tiles first, while the first loads are in flight: each run
     // of masked tiles of a query block is one contiguous slot range per
-    // token, written by all epilogue threads with 16-byte stores.
+    // token, written with 16-byte stores. The block's rows go to different
+    // warps (kEPI / ntok warps a row when there are fewer rows than warps), so
+    // that the stores of all rows are in flight together: a row's stores take
+    // a fixed time of their own, which one warp walking the rows in turn paid
+    // once per row.
     if (R.f_count > 0) {
       QBlk q;
       int j = R.f_j;
       make_qb(P, tqt, R.f_seq, R.f_b, R.f_seqoff, q);
-      const int et = epi * 32 + lane;
       int64_t left = R.f_count;
       while (left > 0) {
         const int64_t seg = min64(left, q.ntr - j);
         const int64_t lo = static_cast<int64_t>(j) * kBlockM;
         const int64_t hi = min64(static_cast<int64_t>(j + seg) * kBlockM, q.row_len);
-        for (int i = 0; i < q.ntok; ++i)
-          fill_mask(p.scores + q.out0 + i * q.row_len, lo, hi, et, kEPI * 32);
+        const int ntok = q.ntok;
+        const int wpr = kEPI / ntok > 1 ? kEPI / ntok : 1;   // warps per row
+        const int ngrp = kEPI / wpr;                          // >= ntok
+        float *const rows = p.scores + q.out0;
+        const int64_t row_len = q.row_len;
+        for (int i = epi / wpr; i < ntok; i += ngrp)
+          fill_mask(rows + i * row_len, lo, hi, (epi % wpr) * 32 + lane, wpr * 32);
         left -= seg;
         if (left > 0) {
           do {

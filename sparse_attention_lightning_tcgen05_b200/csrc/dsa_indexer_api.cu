@@ -15,6 +15,7 @@
 #include "dsa_launch.h"
 #include "score_kernel.cuh"
 #include "topk_cluster.cuh"
+#include "topk_rows.cuh"
 #include "topk_kernel.cuh"
 
 namespace dsa_host {
@@ -369,6 +370,18 @@ dsa_status_t launch_score(const dsa_indexer_desc_t *d, const void *q, const uint
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
+// The row top-k: one CTA per row, a buffer of NT*KPT floats.
+template <int NT, int KPT>
+dsa_status_t launch_topk_rows(DeviceInfo *dev, int which, int T, const TopkParams &p,
+                              cudaStream_t stream) {
+  auto kernel = dsa::topk_rows_kernel<NT, KPT>;
+  const int smem = NT * KPT * 4;
+  dsa_status_t st = ensure_smem_attr(dev, 16 + which, kernel, smem);
+  if (st != DSA_OK) return st;
+  if (launch_pdl(kernel, T, NT, smem, stream, 0, p) != cudaSuccess) return DSA_ERR_CUDA;
+  return DSA_OK;
+}
+
 dsa_status_t launch_topk(const dsa_indexer_desc_t *d, const float *scores,
                          const int32_t *positions, int32_t *topk, cudaStream_t stream) {
   DeviceInfo *dev = nullptr;
@@ -385,10 +398,17 @@ dsa_status_t launch_topk(const dsa_indexer_desc_t *d, const float *scores,
   p.scores = scores;
   p.topk = topk;
   p.k = d->index_topk;
-  // Decode rows are few and long: a cluster of C CTAs per row (up to 8, about
-  // 4096 slots each), the row staged across their shared memories. Prefill
-  // rows are many: 512 threads a row and a smaller stage, so that several
-  // rows run on each SM.
+  // Decode-style rows of at most 4096 slots (pooled keys, short caches): one
+  // CTA a row, the row held in registers. Longer decode rows are few and
+  // long: a cluster of C CTAs per row (up to 8, about 4096 slots each), the
+  // row staged across their shared memories. Prefill rows are many: 512
+  // threads a row and a smaller stage, so that several rows run on each SM.
+  if (p.mode == dsa::kModePositions && d->S <= 4096) {
+    const dsa_status_t rs = d->S <= 2048 ? launch_topk_rows<256, 8>(dev, 0, d->T, p, stream)
+                                         : launch_topk_rows<256, 16>(dev, 1, d->T, p, stream);
+    if (rs != DSA_OK) return rs;
+    return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+  }
   if (p.mode == dsa::kModePositions) {
     using Sh = dsa::ClusterTopkShared<512>;
     const int C = static_cast<int>(std::min<int64_t>(dsa::kClusterMaxRanks,

@@ -201,6 +201,28 @@ __device__ __noinline__ void mbar_drain(uint64_t *bar, uint32_t parity,
   }
 }
 
+// ---- per-thread asynchronous copies global -> shared (cp.async) -------------
+// The issuing thread alone waits for them (cp.async.wait_group) and reads the
+// destination; no other thread's barrier is involved.
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)),
+               "l"(gmem_src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async4(void *smem_dst, const void *gmem_src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)),
+               "l"(gmem_src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// Wait until at most N of this thread's committed groups are in flight.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // ---- TMA (cp.async.bulk.tensor, CTA-local destination, no multicast) ---------
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {

@@ -182,6 +182,49 @@ __device__ __forceinline__ float key_value(uint32_t key) {
   return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
 }
 
+// Row t's scores and its valid length: POSITIONS rows of S slots (valid up to
+// the position, or the compressed rule's last pooled slot); CAUSAL rows of
+// their sequence's L x L block (valid up to the diagonal). All threads of the
+// block call it (CAUSAL synchronises).
+template <int NT, typename SM>
+__device__ __forceinline__ void topk_row_geometry(const TopkParams &p, int t, SM &sm,
+                                                  const float *&row, int64_t &nvalid) {
+  const int tid = threadIdx.x;
+  if (p.mode == kModePositions) {
+    row = p.scores + static_cast<int64_t>(t) * p.S;
+    const int64_t pos = p.compressed ? compressed_last_slot(p.comp, t) : __ldg(p.positions + t);
+    nvalid = pos < 0 ? 0 : (pos + 1 < p.S ? pos + 1 : p.S);
+    return;
+  }
+  if (tid == 0) {            // largest i with cu[i] <= t (cu non-decreasing)
+    int lo = 0, hi = p.num_seqs - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) / 2;
+      if (__ldg(p.cu_seqlens + mid) <= t) lo = mid; else hi = mid - 1;
+    }
+    sm.seq = lo;
+    sm.seq_off = 0;
+  }
+  __syncthreads();
+  const int i = sm.seq;
+  // sum_{j < i} L_j^2: strided over threads, reduced per warp, then summed
+  long long part = 0;
+  for (int j = tid; j < i; j += NT) {
+    const long long L = __ldg(p.cu_seqlens + j + 1) - __ldg(p.cu_seqlens + j);
+    part += L * L;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+  if ((tid & 31) == 0 && part)
+    atomicAdd(reinterpret_cast<unsigned long long *>(&sm.seq_off),
+              static_cast<unsigned long long>(part));
+  __syncthreads();
+  const int a = __ldg(p.cu_seqlens + i);
+  const int64_t L = __ldg(p.cu_seqlens + i + 1) - a;
+  row = p.scores + sm.seq_off + static_cast<int64_t>(t - a) * L;
+  nvalid = t - a + 1;
+}
+
 // Stage the row's values [0, n) in shared memory (if keys != nullptr) and
 // find the smallest and largest key. Vector loads on the 16-byte aligned body.
 template <int NT>
@@ -234,42 +277,9 @@ __global__ void __launch_bounds__(NT) topk_kernel(const TopkParams p) {
   grid_dep_wait();
   grid_dep_launch_dependents();
 
-  // ---- row geometry ----
   const float *row;
   int64_t nvalid;
-  if (p.mode == kModePositions) {
-    row = p.scores + static_cast<int64_t>(t) * p.S;
-    const int64_t pos = p.compressed ? compressed_last_slot(p.comp, t) : __ldg(p.positions + t);
-    nvalid = pos < 0 ? 0 : (pos + 1 < p.S ? pos + 1 : p.S);
-  } else {
-    if (tid == 0) {            // largest i with cu[i] <= t (cu non-decreasing)
-      int lo = 0, hi = p.num_seqs - 1;
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) / 2;
-        if (__ldg(p.cu_seqlens + mid) <= t) lo = mid; else hi = mid - 1;
-      }
-      sm.seq = lo;
-      sm.seq_off = 0;
-    }
-    __syncthreads();
-    const int i = sm.seq;
-    // sum_{j < i} L_j^2: strided over threads, reduced per warp, then summed
-    long long part = 0;
-    for (int j = tid; j < i; j += NT) {
-      const long long L = __ldg(p.cu_seqlens + j + 1) - __ldg(p.cu_seqlens + j);
-      part += L * L;
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-    if ((tid & 31) == 0 && part)
-      atomicAdd(reinterpret_cast<unsigned long long *>(&sm.seq_off),
-                static_cast<unsigned long long>(part));
-    __syncthreads();
-    const int a = __ldg(p.cu_seqlens + i);
-    const int64_t L = __ldg(p.cu_seqlens + i + 1) - a;
-    row = p.scores + sm.seq_off + static_cast<int64_t>(t - a) * L;
-    nvalid = t - a + 1;
-  }
+  topk_row_geometry<NT>(p, t, sm, row, nvalid);
   int *out = p.topk + static_cast<int64_t>(t) * p.k;
   const uint32_t k = static_cast<uint32_t>(p.k);
 

@@ -247,3 +247,31 @@ def test_c4_prefill_full_size_sampled(dsa):
     rows = sorted(set([0, 2, 3, 4, 511, 4095, 4096, 8190, 8191] +
                       list(rng.integers(0, wl.T, 12))))
     run_and_check(dsa, wl, syn.generate(wl), rows=rows)
+
+
+# ---- top-k of short decode-style rows (the register path) -------------------
+
+def test_decode_topk_ties_integer_scores(dsa):
+    """H=1 integer inputs: many equal scores around the threshold; the set
+    must be the oracle's, lower slots first among ties (bit-exact)."""
+    wl = decode_wl(T=24, H=1, S=2000, k=300, shared=True, pos=(400, 2000), seed=60)
+    run_and_check(dsa, wl, syn.generate(wl, value_kind="int"), exact=True)
+
+
+def test_decode_topk_all_scores_equal(dsa):
+    """Every score 0 (q = 0): the threshold's ties fill the whole set, which
+    must be the lowest k slots of each row."""
+    wl = decode_wl(T=6, H=64, S=3000, k=700, shared=True, pos=(800, 3000), seed=61)
+    inputs = syn.generate(wl)
+    inputs["q"] = np.zeros_like(inputs["q"])
+    run_and_check(dsa, wl, inputs, exact=True)
+
+
+@pytest.mark.parametrize("S", [33, 2048, 2049, 4096])
+def test_decode_topk_row_lengths(dsa, S):
+    """Rows at the register path's boundaries (one and two chunk rows, the
+    largest rows it takes) and a misaligned row start (S odd)."""
+    wl = decode_wl(T=5, H=16, S=S, k=min(32, S - 1), shared=True, pos=(0, S), seed=62)
+    inputs = syn.generate(wl)
+    inputs["positions"] = np.array([S - 1, S // 2, 31, 32, S + 5], np.int32)
+    run_and_check(dsa, wl, inputs)

@@ -56,6 +56,21 @@ class Workload:
     seed: int = 0
     query_start: int = 0           # COMPRESSED: absolute position of query 0
     compress_ratio: int = 0        # COMPRESSED: tokens pooled per slot
+    page_size: int = 0             # POSITIONS, one cache per token: > 0 = paged cache
+
+    @property
+    def paged(self) -> bool:
+        return self.mode == MODE_POSITIONS and not self.shared_cache and self.page_size > 0
+
+    @property
+    def pages_per_seq(self) -> int:
+        """Block-table entries per token (paged caches)."""
+        return -(-self.S // self.page_size) if self.paged else 0
+
+    @property
+    def num_pages(self) -> int:
+        """Pages in the pool (paged caches): exactly the pages the tokens use."""
+        return self.T * self.pages_per_seq
 
     @property
     def num_seqs(self) -> int:
@@ -67,15 +82,18 @@ class Workload:
 
     @property
     def key_slots(self) -> int:
-        """Rows of the key cache buffer (slots of all sequences)."""
+        """Rows of the key cache buffer (slots of all sequences; paged: of
+        all pages)."""
         if self.mode == MODE_CAUSAL:
             return int(sum(self.seqlens))
+        if self.paged:
+            return self.num_pages * self.page_size
         return self.S * self.num_seqs
 
     @property
     def k_seq_stride(self) -> int:
         """Elements between consecutive sequences' caches (POSITIONS)."""
-        if self.mode != MODE_POSITIONS or self.shared_cache:
+        if self.mode != MODE_POSITIONS or self.shared_cache or self.paged:
             return 0
         return self.S * self.D
 
@@ -219,7 +237,11 @@ def generate(wl: Workload, value_kind: str = "gauss",
     q_scale ([T,H,D/32] uint8 or None), k ([key_slots, D]), k_scale, w
     ([T,H] float32), positions ([T] int32, POSITIONS only), cu_seqlens
     ([num_seqs+1] int32, CAUSAL only). COMPRESSED draws neither: validity
-    follows from query_start and compress_ratio.
+    follows from query_start and compress_ratio. A paged cache (page_size >
+    0) draws k as a pool of num_pages pages ([num_pages*page_size, D]) and,
+    after the positions, block_table ([T, pages_per_seq] int32): a random
+    permutation of the page ids, so that each token's pages are scattered
+    over the pool.
     """
     rng = np.random.default_rng(wl.seed if seed is None else seed)
     T, H, D = wl.T, wl.H, wl.D
@@ -234,10 +256,13 @@ def generate(wl: Workload, value_kind: str = "gauss",
     else:
         w = (gaussian_f32(rng, T * H) * np.float32(wl.w_scale)).reshape(T, H)
     out = dict(q=q, q_scale=q_scale, k=k, k_scale=k_scale, w=w,
-               positions=None, cu_seqlens=None)
+               positions=None, cu_seqlens=None, block_table=None)
     if wl.mode == MODE_POSITIONS:
         out["positions"] = rng.integers(wl.pos_lo, wl.pos_hi, size=T,
                                         dtype=np.int32)
+        if wl.paged:
+            out["block_table"] = rng.permutation(wl.num_pages).astype(
+                np.int32).reshape(T, wl.pages_per_seq)
     elif wl.mode == MODE_CAUSAL:
         out["cu_seqlens"] = wl.cu_seqlens()
     return out

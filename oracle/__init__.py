@@ -45,7 +45,9 @@ class _Problem(ctypes.Structure):
                 ("q", ctypes.c_void_p), ("q_scale", ctypes.c_void_p),
                 ("w", ctypes.c_void_p), ("k", ctypes.c_void_p),
                 ("k_scale", ctypes.c_void_p), ("query_start", ctypes.c_int64),
-                ("compress_ratio", ctypes.c_int32), ("pad_", ctypes.c_int32)]
+                ("compress_ratio", ctypes.c_int32), ("page_size", ctypes.c_int32),
+                ("pages_per_seq", ctypes.c_int32), ("num_pages", ctypes.c_int32),
+                ("block_table", ctypes.c_void_p)]
 
 
 _lib = None
@@ -103,7 +105,14 @@ class Problem:
             q=_ptr(a["q"]), q_scale=_ptr(a.get("q_scale")),
             w=_ptr(a["w"]),
             k=_ptr(a["k"]), k_scale=_ptr(a.get("k_scale")),
-            query_start=wl.query_start, compress_ratio=wl.compress_ratio)
+            query_start=wl.query_start, compress_ratio=wl.compress_ratio,
+            page_size=wl.page_size if wl.paged else 0,
+            pages_per_seq=wl.pages_per_seq, num_pages=wl.num_pages,
+            block_table=_ptr(a.get("block_table")))
+        if wl.paged:
+            bt = a["block_table"]
+            assert bt is not None and bt.dtype == np.int32
+            assert bt.shape == (wl.T, wl.pages_per_seq)
 
     def row_info(self, t: int):
         """(first_slot, row_len, last_valid, score_offset) of query row t."""

@@ -28,6 +28,10 @@
  *    mathematical no-op for the score; scales are block-32 e8m0 (qr_scale_hbm).
  *  - NeMo AutoModel optimized_kernels, sparse_attention_torch parameters:
  *    a top-k index of -1 masks an entry.
+ *  - tokamax Supported Ops, lightning_indexer: the scores run over a paged
+ *    KV cache. Reading: token t's cache slot s lives in page
+ *    block_table[t][s / page_size], at row s % page_size of it; the pages
+ *    form one pool [num_pages, page_size, D] (and [.., D/32] scales).
  *  - NeMo AutoModel optimized_kernels, dsv4_indexer_scores: the compressed
  *    (C4) indexer scores queries against pooled_kv, keys pooled over
  *    compress_ratio consecutive tokens, for a query chunk that starts at
@@ -85,7 +89,10 @@ typedef struct {
     const uint8_t *k_scale;     /* [slots, D/32] e8m0 (FP8) */
     int64_t query_start;        /* COMPRESSED: absolute position of query 0 */
     int32_t compress_ratio;     /* COMPRESSED: tokens pooled per slot (>= 1) */
-    int32_t pad_;
+    int32_t page_size;          /* POSITIONS, paged cache: slots per page */
+    int32_t pages_per_seq;      /* paged: block-table entries per token */
+    int32_t num_pages;          /* paged: pages in the pool k / k_scale */
+    const int32_t *block_table; /* paged: [T, pages_per_seq] page ids; NULL = not paged */
 } orc_problem;
 
 /* ---- exact decoding of the storage formats -------------------------------- */
@@ -147,7 +154,8 @@ int orc_row_info(const orc_problem *p, int64_t t, int64_t *first_slot,
     if (t < 0 || t >= p->T)
         return -1;
     if (p->mode == ORC_MODE_POSITIONS) {
-        *first_slot = t * (p->k_seq_stride / p->D);
+        /* a paged cache addresses its slots through the block table */
+        *first_slot = p->block_table ? 0 : t * (p->k_seq_stride / p->D);
         *row_len = p->S;
         *last_valid = p->positions[t];          /* s <= positions[t] */
         *score_offset = t * p->S;
@@ -176,6 +184,17 @@ int orc_row_info(const orc_problem *p, int64_t t, int64_t *first_slot,
     return -1;
 }
 
+/* Row of the k array holding slot s of token t's cache (first: the row of
+ * slot 0, from orc_row_info): the slot itself, or with a block table (paged
+ * cache) row s % page_size of page block_table[t][s / page_size]. */
+static int64_t key_row(const orc_problem *p, int64_t t, int64_t first, int64_t s)
+{
+    if (!p->block_table)
+        return first + s;
+    int64_t page = p->block_table[t * p->pages_per_seq + s / p->page_size];
+    return page * p->page_size + s % p->page_size;
+}
+
 /* Score row of query token t into out[0 .. row_len). */
 static void score_row(const orc_problem *p, int64_t t, double *out,
                       double *qrow, double *krow)
@@ -193,7 +212,8 @@ static void score_row(const orc_problem *p, int64_t t, double *out,
             continue;
         }
         for (int32_t d = 0; d < D; ++d)
-            krow[d] = stored_value(p->dtype, p->k, p->k_scale, first + s, D, d);
+            krow[d] = stored_value(p->dtype, p->k, p->k_scale, key_row(p, t, first, s),
+                                   D, d);
         double I = 0.0;
         for (int32_t h = 0; h < H; ++h) {
             double x = 0.0;                     /* q[t,h,:] . k[s,:] */

@@ -5,6 +5,7 @@ hand-worked golden rows, brute-force sorts, a BLAS matmul, linear identities
 that the ReLU and the head weights must satisfy, the Hadamard identity, exact
 integer arithmetic and the library's e4m3 decoding table.
 """
+import dataclasses
 import json
 import os
 
@@ -366,6 +367,77 @@ def test_compressed_equals_shared_cache_positions(dtype):
             got = tk[t].tolist()
             assert got[n:] == [-1] * (k - n)
             assert sorted(got[:n]) == sorted(_brute_topk(sc[t], int(last[t]), k)[:n])
+
+
+def _small_paged(T=6, H=4, S=300, page=64, seed=7, dtype=syn.DTYPE_BF16):
+    wl = syn.Workload("pg", syn.MODE_POSITIONS, T=T, H=H, D=128, index_topk=16,
+                      S=S, pos_lo=0, pos_hi=S, page_size=page, dtype=dtype,
+                      w_scale=0.5, seed=seed)
+    return wl, syn.generate(wl)
+
+
+def _gather_pages(wl, inputs, key):
+    """Each token's cache as one dense [S, ...] array, pages taken in block-table
+    order (numpy fancy indexing, no oracle code)."""
+    pool = inputs[key].reshape(wl.num_pages, wl.page_size, -1)
+    return np.concatenate([pool[inputs["block_table"][t]].reshape(-1, pool.shape[-1])[:wl.S]
+                           for t in range(wl.T)])
+
+
+@pytest.mark.parametrize("dtype,page", [(syn.DTYPE_BF16, 64), (syn.DTYPE_BF16, 16),
+                                        (syn.DTYPE_BF16, 128), (syn.DTYPE_FP8, 32)])
+def test_paged_cache_equals_gathered_dense_cache(dtype, page):
+    """A paged cache scores like the dense per-token cache its block table
+    describes (the pages gathered in numpy)."""
+    wl, inputs = _small_paged(page=page, dtype=dtype, S=333)
+    rows = list(range(wl.T))
+    P = oracle.Problem(wl, inputs)
+    sp = P.scores(rows)
+    wd = dataclasses.replace(wl, page_size=0)
+    dense = dict(inputs, k=_gather_pages(wl, inputs, "k"), block_table=None,
+                 k_scale=None if inputs["k_scale"] is None else _gather_pages(wl, inputs, "k_scale"))
+    Pd = oracle.Problem(wd, dense)
+    sd = Pd.scores(rows)
+    for t in rows:
+        np.testing.assert_array_equal(sp[t], sd[t])
+    for k in (1, 16, 400):
+        assert [sorted(x) for x in P.topk(rows, sp, k).tolist()] == \
+               [sorted(x) for x in Pd.topk(rows, sd, k).tolist()]
+
+
+def test_paged_cache_page_permutation_invariance():
+    """Moving the pages within the pool, and the block table with them,
+    changes nothing."""
+    wl, inputs = _small_paged(page=32)
+    rows = list(range(wl.T))
+    base = oracle.Problem(wl, inputs).scores(rows)
+    perm = np.random.default_rng(5).permutation(wl.num_pages)     # new home of page i
+    pool = inputs["k"].reshape(wl.num_pages, wl.page_size, -1)
+    moved = np.empty_like(pool)
+    moved[perm] = pool
+    moved_inputs = dict(inputs, k=moved.reshape(inputs["k"].shape),
+                        block_table=perm[inputs["block_table"]].astype(np.int32))
+    got = oracle.Problem(wl, moved_inputs).scores(rows)
+    for t in rows:
+        np.testing.assert_array_equal(got[t], base[t])
+
+
+def test_paged_cache_reads_only_valid_slots():
+    """Pages (and rows of a token's last page) past its position may hold
+    anything: NaN there changes no score."""
+    wl, inputs = _small_paged(page=16, S=200)
+    rows = list(range(wl.T))
+    base = oracle.Problem(wl, inputs).scores(rows)
+    k = inputs["k"].copy().reshape(wl.num_pages, wl.page_size, -1)
+    for t in rows:
+        pos = int(inputs["positions"][t])
+        for lp, page in enumerate(inputs["block_table"][t]):
+            for r in range(wl.page_size):
+                if lp * wl.page_size + r > pos:
+                    k[page, r] = 0x7FC0                         # a bf16 NaN
+    got = oracle.Problem(wl, dict(inputs, k=k.reshape(inputs["k"].shape))).scores(rows)
+    for t in rows:
+        np.testing.assert_array_equal(got[t], base[t])
 
 
 def test_causal_layout_tiles_packed_buffer():

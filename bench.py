@@ -41,6 +41,7 @@ UNIT = "pairs/s"
 DEFAULTS = {   # steps, warmup, graph length
     "tiny_decode": (100000, 5000, 500),
     "decode_batch": (60000, 3000, 240),
+    "decode_batch_paged": (60000, 3000, 240),
     "long_decode_fp8": (6000, 300, 60),
     "prefill_causal": (1500, 30, 30),
     "ragged_prefill": (20, 3, 1),
@@ -335,9 +336,10 @@ def run_e2e(args, wl, inputs, p, pairs, stream, device, dist):
             a = a.view(np.int16)
         return torch.from_numpy(a).pin_memory()
     host = {k: pinned(inputs.get(k)) for k in ("q", "q_scale", "w", "k", "k_scale",
-                                                "positions", "cu_seqlens")}
+                                                "positions", "cu_seqlens", "block_table")}
     dev = {"q": p.q, "q_scale": p.q_scale, "w": p.w, "k": p.k_cache,
-           "k_scale": p.k_scale, "positions": p.positions, "cu_seqlens": p.cu_seqlens}
+           "k_scale": p.k_scale, "positions": p.positions, "cu_seqlens": p.cu_seqlens,
+           "block_table": p.block_table}
     out_s = torch.empty(p.scores.shape, dtype=p.scores.dtype).pin_memory()
     out_t = torch.empty(p.topk.shape, dtype=p.topk.dtype).pin_memory()
     h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
@@ -459,7 +461,9 @@ def workload_config(wl, extra=None):
                   syn.MODE_COMPRESSED: "compressed"}[wl.mode]}
     if wl.mode == syn.MODE_POSITIONS:
         c.update(S=wl.S, positions=f"U[{wl.pos_lo},{wl.pos_hi})",
-                 caches="shared" if wl.shared_cache else "one per token")
+                 caches="shared" if wl.shared_cache else (
+                     f"one per token, paged ({wl.page_size}-slot pages)" if wl.paged
+                     else "one per token"))
     elif wl.mode == syn.MODE_COMPRESSED:
         c.update(S=wl.S, compress_ratio=wl.compress_ratio, query_start=wl.query_start,
                  caches="one pooled cache")

@@ -121,6 +121,11 @@ WORKLOADS = {
                                D=128, index_topk=2048,
                                seqlens=(4096, 16384, 32768, 65536),
                                w_scale=1.0 / 8.0),
+    # the decode batch over a paged cache (pages of 64 slots, scattered over
+    # the pool by a random block table)
+    "decode_batch_paged": Workload("decode_batch_paged", MODE_POSITIONS, T=16, H=64,
+                                   D=128, index_topk=2048, S=32768, pos_lo=2048,
+                                   pos_hi=32768, w_scale=1.0 / 8.0, page_size=64),
     # compressed (C4) indexer, the next step beyond the five: an 8192-token
     # prefill chunk against its 2048 keys pooled 4:1, DSV4's index_topk 1024
     "c4_prefill": Workload("c4_prefill", MODE_COMPRESSED, T=8192, H=64, D=128,

@@ -28,6 +28,9 @@
  *    Hadamard rotation because it is a no-op for q . k.
  *  - NeMo AutoModel optimized_kernels, sparse_attention_torch: a key index of
  *    -1 masks an entry.
+ *  - tokamax Supported Ops, lightning_indexer: the scores run over a paged
+ *    KV cache. This library reads it as one pool of pages and a block table
+ *    with one row per query token (see block_table below).
  *  - NeMo AutoModel optimized_kernels, dsv4_indexer_scores and
  *    indexer_scores_torch: the DSV4 "C4" indexer scores queries against a
  *    pooled (compressed) key cache, given compress_ratio and query_start.
@@ -121,6 +124,19 @@ typedef struct {
                               Otherwise unused                                  */
   int32_t compress_ratio;  /* COMPRESSED: raw tokens per pooled slot, >= 1.
                               Otherwise unused                                  */
+  int32_t page_size;       /* paged POSITIONS cache (block_table != NULL): slots
+                              per page, a power of two in [16, 65536]            */
+  int32_t pages_per_seq;   /* paged: block-table entries per token, >= 1, with
+                              S <= pages_per_seq * page_size                    */
+  int32_t num_pages;       /* paged: pages in the pool k points to, >= 1        */
+  const int32_t *block_table; /* NULL: not paged. Paged (POSITIONS, bf16 only,
+                              k_seq_stride 0): device [T, pages_per_seq] int32;
+                              token t's slot s is row s % page_size of page
+                              block_table[t*pages_per_seq + s/page_size] of the
+                              pool k [num_pages, page_size, D]. Entries of pages
+                              that hold a valid slot must lie in
+                              [0, num_pages); other entries are never used for
+                              a score (a page id outside the pool reads as 0)  */
 } dsa_indexer_desc_t;
 
 /*
@@ -128,7 +144,8 @@ typedef struct {
  *  q        [T, H, D]      bf16, or e4m3 bytes                 (16-byte aligned)
  *  q_scale  [T, H, D/32]   e8m0 bytes (FP8 only; NULL for BF16)
  *  w        [T, H]         fp32
- *  k        POSITIONS: cache of token t at element t*k_seq_stride, [S, D]
+ *  k        POSITIONS: cache of token t at element t*k_seq_stride, [S, D];
+ *           paged: the page pool [num_pages, page_size, D]
  *           COMPRESSED: the pooled cache [S, D]
  *           CAUSAL:    [T, D], sequence i at rows cu[i] .. cu[i+1]-1
  *           bf16, or e4m3 bytes                                 (16-byte aligned)

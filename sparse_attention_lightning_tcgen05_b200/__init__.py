@@ -42,7 +42,9 @@ class dsa_indexer_desc_t(ctypes.Structure):
                 ("S", ctypes.c_int64), ("k_seq_stride", ctypes.c_int64),
                 ("num_seqs", ctypes.c_int32), ("cu_seqlens", ctypes.c_void_p),
                 ("dtype", ctypes.c_int), ("mask", ctypes.c_int),
-                ("query_start", ctypes.c_int64), ("compress_ratio", ctypes.c_int32)]
+                ("query_start", ctypes.c_int64), ("compress_ratio", ctypes.c_int32),
+                ("page_size", ctypes.c_int32), ("pages_per_seq", ctypes.c_int32),
+                ("num_pages", ctypes.c_int32), ("block_table", ctypes.c_void_p)]
 
 
 class DsaError(RuntimeError):
@@ -84,12 +86,15 @@ def _ptr(x) -> int | None:
 
 def make_desc(T, H, index_topk, *, D=128, S=0, k_seq_stride=0, num_seqs=0,
               cu_seqlens=None, dtype=DSA_KV_BF16, mask=DSA_MASK_POSITIONS,
-              query_start=0, compress_ratio=0):
+              query_start=0, compress_ratio=0, page_size=0, pages_per_seq=0,
+              num_pages=0, block_table=None):
     return dsa_indexer_desc_t(T=T, H=H, D=D, index_topk=index_topk, S=S,
                               k_seq_stride=k_seq_stride, num_seqs=num_seqs,
                               cu_seqlens=_ptr(cu_seqlens), dtype=dtype,
                               mask=mask, query_start=query_start,
-                              compress_ratio=compress_ratio)
+                              compress_ratio=compress_ratio, page_size=page_size,
+                              pages_per_seq=pages_per_seq, num_pages=num_pages,
+                              block_table=_ptr(block_table))
 
 
 def dsa_status_string(status: int) -> str:

@@ -105,6 +105,17 @@ dsa_status_t check_desc(const dsa_indexer_desc_t *d) {
   if (d->D != 128) return DSA_ERR_UNSUPPORTED;
   if (d->H > 256) return DSA_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(d->T) * d->H > INT32_MAX - 256) return DSA_ERR_UNSUPPORTED;
+  if (d->block_table) {
+    // a paged cache: one page pool, a block-table row per token
+    if (d->mask != DSA_MASK_POSITIONS || d->k_seq_stride != 0) return DSA_ERR_INVALID_ARG;
+    if (d->page_size < 16 || d->page_size > 65536 || (d->page_size & (d->page_size - 1)) != 0)
+      return DSA_ERR_INVALID_ARG;
+    if (d->pages_per_seq < 1 || d->num_pages < 1) return DSA_ERR_INVALID_ARG;
+    if (d->S < 1 || d->S > static_cast<int64_t>(d->pages_per_seq) * d->page_size)
+      return DSA_ERR_INVALID_ARG;
+    if (!aligned(d->block_table, 4)) return DSA_ERR_INVALID_ARG;
+    if (d->dtype != DSA_KV_BF16) return DSA_ERR_UNSUPPORTED;
+  }
   if (d->mask == DSA_MASK_POSITIONS) {
     if (d->S < 1) return DSA_ERR_INVALID_ARG;
     if (d->S > INT32_MAX - 256) return DSA_ERR_UNSUPPORTED;
@@ -232,7 +243,7 @@ ScoreLaunch choose_score_compressed(const dsa_indexer_desc_t *d) {
 ScoreLaunch choose_score(const dsa_indexer_desc_t *d) {
   if (d->mask == DSA_MASK_COMPRESSED) return choose_score_compressed(d);
   const bool causal = d->mask == DSA_MASK_CAUSAL;
-  const bool per_token_cache = !causal && d->k_seq_stride != 0;
+  const bool per_token_cache = !causal && (d->k_seq_stride != 0 || d->block_table);
   const int H = d->H;
   if (d->dtype == DSA_KV_BF16) {
     if (per_token_cache) {
@@ -288,7 +299,8 @@ dsa_status_t launch_score(const dsa_indexer_desc_t *d, const void *q, const uint
   if (st != DSA_OK) return st;
 
   const bool causal = d->mask == DSA_MASK_CAUSAL;
-  const bool shared = causal || d->k_seq_stride == 0;
+  const bool paged = d->block_table != nullptr;
+  const bool shared = causal || (d->k_seq_stride == 0 && !paged);
   const cuuint64_t rows = causal ? static_cast<cuuint64_t>(d->T) : static_cast<cuuint64_t>(d->S);
   const cuuint64_t caches = shared ? 1 : static_cast<cuuint64_t>(d->T);
   const cuuint64_t elt = L.fp8 ? 1 : 2;
@@ -297,7 +309,17 @@ dsa_status_t launch_score(const dsa_indexer_desc_t *d, const void *q, const uint
   CUtensorMap tk, tq, tksf, tqsf;
   std::memset(&tksf, 0, sizeof tksf);
   std::memset(&tqsf, 0, sizeof tqsf);
-  {
+  if (paged) {
+    // the page pool: [num_pages, page_size, D]; a 128-slot key tile is one
+    // box (pages of >= 128 slots) or 128/page_size boxes of one page each
+    const cuuint64_t ps = static_cast<cuuint64_t>(d->page_size);
+    const cuuint64_t dims[3] = {128, ps, static_cast<cuuint64_t>(d->num_pages)};
+    const cuuint64_t strides[2] = {128 * elt, ps * 128 * elt};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elt),
+                               static_cast<cuuint32_t>(std::min<cuuint64_t>(ps, dsa::kBlockM)), 1};
+    st = make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, k, dims, strides, box);
+    if (st != DSA_OK) return st;
+  } else {
     const cuuint64_t dims[3] = {128, rows, caches};
     const cuuint64_t strides[2] = {128 * elt, stride_elems * elt};
     const cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elt), dsa::kBlockM, 1};
@@ -337,7 +359,11 @@ dsa_status_t launch_score(const dsa_indexer_desc_t *d, const void *q, const uint
   p.T = d->T;
   p.H = d->H;
   p.S = d->S;
-  p.shared_cache = d->k_seq_stride == 0;
+  p.shared_cache = shared;
+  p.block_table = d->block_table;
+  p.pages_per_seq = paged ? d->pages_per_seq : 0;
+  p.num_pages = paged ? d->num_pages : 0;
+  p.page_shift = paged ? __builtin_ctz(static_cast<unsigned>(d->page_size)) : 0;
   p.num_seqs = d->num_seqs;
   p.cu_seqlens = d->cu_seqlens;
   // COMPRESSED runs as POSITIONS over one shared cache, with no positions

@@ -55,6 +55,10 @@ struct ScoreParams {
   int T, H;
   int64_t S;                 // POSITIONS: slots per cache
   int shared_cache;          // POSITIONS: every token reads cache 0
+  const int *block_table;    // POSITIONS, paged: [T, pages_per_seq] page ids (else NULL)
+  int pages_per_seq;         // paged: block-table entries per token
+  int num_pages;             // paged: pages in the pool (an id past it reads as zeros)
+  int page_shift;            // paged: log2(slots per page)
   int num_seqs;              // CAUSAL
   const int *cu_seqlens;     // CAUSAL
   const int *positions;      // POSITIONS
@@ -788,6 +792,24 @@ __global__ void __launch_bounds__((2 + kEPI + (kFP8 ? 1 : 0) + (kISS - 1)) * 32,
         for (int i = 0; i < g; ++i) {
           uint8_t *dst = sk + (st.idx * kG + i) * L.k_stage_bytes;
           const int y = c.q.y0 + (c.j + i) * kBlockM;
+          if (!kFP8 && p.block_table) {
+            // paged cache: the tile's slots y .. y+127 from one page, or from
+            // 128/page_size pages (one box each, at its row offset in the
+            // tile; 128-byte swizzle atoms are 8 rows, boxes >= 16 rows).
+            // Past the block table, an id past the pool: TMA fills zeros.
+            const int box = p.page_shift >= 7 ? kBlockM : (1 << p.page_shift);
+            for (int b = 0; b < kBlockM; b += box) {
+              const int lp = (y + b) >> p.page_shift;
+              const int row = (y + b) & ((1 << p.page_shift) - 1);
+              const int page =
+                  lp < p.pages_per_seq
+                      ? __ldg(p.block_table + static_cast<int64_t>(c.q.z) * p.pages_per_seq + lp)
+                      : p.num_pages;
+              tma_load_3d(dst + b * 128, &tmap_k, full_k + st.idx, 0, row, page);
+              tma_load_3d(dst + kBlockM * 128 + b * 128, &tmap_k, full_k + st.idx, 64, row, page);
+            }
+            continue;
+          }
           tma_load_3d(dst, &tmap_k, full_k + st.idx, 0, y, c.q.z);
           if constexpr (kFP8) {
             tma_load_2d(sksf + (st.idx * kG + i) * L.k_sf_bytes, &tmap_ksf, full_k + st.idx,

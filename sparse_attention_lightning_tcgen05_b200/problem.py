@@ -31,7 +31,7 @@ class DeviceProblem:
     def __init__(self, *, mode, T, H, index_topk, q, w, k, dtype=DSA_KV_BF16,
                  S=0, k_seq_stride=0, cu_seqlens=None, positions=None,
                  q_scale=None, k_scale=None, query_start=0, compress_ratio=0,
-                 device="cuda"):
+                 page_size=0, block_table=None, num_pages=0, device="cuda"):
         self.mode, self.T, self.H, self.k = mode, T, H, index_topk
         self.S, self.dtype = S, dtype
         self.q = _dev(q, device)
@@ -41,6 +41,7 @@ class DeviceProblem:
         self.k_scale = _dev(k_scale, device)
         self.positions = _dev(positions, device)
         self.cu_seqlens = _dev(cu_seqlens, device)
+        self.block_table = _dev(block_table, device)
         if mode == DSA_MASK_CAUSAL:
             cu = np.asarray(cu_seqlens if not isinstance(cu_seqlens, torch.Tensor)
                             else cu_seqlens.cpu().numpy(), np.int64)
@@ -53,7 +54,10 @@ class DeviceProblem:
         self.desc = make_desc(T, H, index_topk, S=S, k_seq_stride=k_seq_stride,
                               num_seqs=self.num_seqs, cu_seqlens=self.cu_seqlens,
                               dtype=dtype, mask=mode, query_start=query_start,
-                              compress_ratio=compress_ratio)
+                              compress_ratio=compress_ratio, page_size=page_size,
+                              pages_per_seq=(0 if block_table is None
+                                             else int(block_table.shape[1])),
+                              num_pages=num_pages, block_table=self.block_table)
         self.scores = torch.empty(n_scores, dtype=torch.float32, device=device)
         self.topk = torch.empty((T, index_topk), dtype=torch.int32, device=device)
         self.ws_bytes = dsa_indexer_workspace_size(self.desc)
@@ -71,6 +75,8 @@ class DeviceProblem:
                    positions=inputs.get("positions"),
                    q_scale=inputs.get("q_scale"), k_scale=inputs.get("k_scale"),
                    query_start=wl.query_start, compress_ratio=wl.compress_ratio,
+                   page_size=wl.page_size if wl.paged else 0,
+                   block_table=inputs.get("block_table"), num_pages=wl.num_pages,
                    device=device)
 
     def _stream(self, stream):

@@ -97,6 +97,38 @@ def test_bad_compressed_descriptors(kw, code):
     assert e.value.status == code
 
 
+def paged_desc(**kw):
+    d = dict(T=4, H=64, index_topk=16, S=1000, k_seq_stride=0, page_size=64,
+             pages_per_seq=16, num_pages=64, block_table=1 << 20)
+    d.update(kw)
+    return dsa.make_desc(**d)
+
+
+def test_paged_descriptor_layout():
+    f = dsa.dsa_indexer_desc_t
+    assert f.page_size.offset == f.compress_ratio.offset + 4
+    assert f.block_table.offset % 8 == 0 and f.block_table.offset == f.num_pages.offset + 4
+    assert dsa.dsa_indexer_workspace_size(paged_desc()) >= 256
+    assert dsa.dsa_indexer_workspace_size(paged_desc(page_size=16, pages_per_seq=63)) >= 256
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(page_size=48), dsa.DSA_ERR_INVALID_ARG),            # not a power of two
+    (dict(page_size=8, pages_per_seq=125), dsa.DSA_ERR_INVALID_ARG),   # below 16
+    (dict(page_size=1 << 17, pages_per_seq=1), dsa.DSA_ERR_INVALID_ARG),
+    (dict(pages_per_seq=15), dsa.DSA_ERR_INVALID_ARG),          # S > 15 * 64
+    (dict(num_pages=0), dsa.DSA_ERR_INVALID_ARG),
+    (dict(k_seq_stride=1000 * 128), dsa.DSA_ERR_INVALID_ARG),   # a pool, not per-token caches
+    (dict(mask=dsa.DSA_MASK_CAUSAL, num_seqs=1, cu_seqlens=1 << 20), dsa.DSA_ERR_INVALID_ARG),
+    (dict(block_table=(1 << 20) + 2), dsa.DSA_ERR_INVALID_ARG),   # misaligned table
+    (dict(dtype=dsa.DSA_KV_FP8_E4M3_E8M0_B32), dsa.DSA_ERR_UNSUPPORTED),
+])
+def test_bad_paged_descriptors(kw, code):
+    with pytest.raises(dsa.DsaError) as e:
+        dsa.dsa_indexer_workspace_size(paged_desc(**kw))
+    assert e.value.status == code
+
+
 def test_compressed_rejects_a_positions_array():
     d = compressed_desc()
     fake = 1 << 20

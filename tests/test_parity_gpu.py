@@ -275,3 +275,47 @@ def test_decode_topk_row_lengths(dsa, S):
     inputs = syn.generate(wl)
     inputs["positions"] = np.array([S - 1, S // 2, 31, 32, S + 5], np.int32)
     run_and_check(dsa, wl, inputs)
+
+
+# ---- paged key caches (block tables) ------------------------------------------
+
+def paged_wl(T, H, S, k, page, seed=0):
+    return syn.Workload("pg", syn.MODE_POSITIONS, T=T, H=H, D=128, index_topk=k, S=S,
+                        pos_lo=0, pos_hi=S, page_size=page,
+                        w_scale=1.0 / np.sqrt(H), seed=seed)
+
+
+@pytest.mark.parametrize("page", [16, 32, 64, 128, 256])
+def test_paged_decode(dsa, page):
+    """Pages smaller than a key tile (several pages a tile), equal to it and
+    larger; S not a multiple of the page."""
+    wl = paged_wl(T=5, H=64, S=1000, k=64, page=page, seed=70 + page)
+    run_and_check(dsa, wl, syn.generate(wl))
+
+
+def test_paged_decode_integer_bit_exact(dsa):
+    wl = paged_wl(T=4, H=64, S=700, k=40, page=32, seed=71)
+    run_and_check(dsa, wl, syn.generate(wl, value_kind="int"), exact=True)
+
+
+def test_paged_generic_heads(dsa):
+    wl = paged_wl(T=6, H=4, S=900, k=50, page=64, seed=72)
+    run_and_check(dsa, wl, syn.generate(wl))
+
+
+def test_paged_unused_table_entries(dsa):
+    """Block-table entries of pages past a token's position may be anything
+    (-1, past the pool): the scores of the valid slots do not change."""
+    wl = paged_wl(T=6, H=64, S=1200, k=64, page=64, seed=73)
+    inputs = syn.generate(wl)
+    inputs["positions"] = np.array([0, 63, 64, 500, 1199, 129], np.int32)
+    bt = inputs["block_table"].copy()
+    for t, pos in enumerate(inputs["positions"]):
+        bt[t, pos // 64 + 1:] = np.where(np.arange(bt.shape[1] - pos // 64 - 1) % 2, -1, 1 << 30)
+    inputs["block_table"] = bt
+    run_and_check(dsa, wl, inputs)
+
+
+def test_decode_batch_paged_full_size(dsa):
+    wl = syn.WORKLOADS["decode_batch_paged"]
+    run_and_check(dsa, wl, syn.generate(wl))

@@ -600,6 +600,46 @@ __device__ __forceinline__ float head_sum_h64(uint32_t taddr, const float *wrow)
          ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
 }
 
+// The same head sums for the tokens [i_lo, i_hi) of one accumulator (64
+// columns a token; w rows at wsh, 64 floats each), with the next 32-column
+// TMEM load in flight while the current one is reduced: one load is
+// outstanding at a time, so each wait covers exactly the load it needs. The
+// sums are formed in the same order as head_sum_h64. store(i, sum).
+template <typename Store>
+__device__ __forceinline__ void head_sums_h64_pipelined(uint32_t tbase, int i_lo, int i_hi,
+                                                        const float *wsh, Store store) {
+  if (i_lo >= i_hi) return;
+  float ra[32], rb[32];
+  tmem_ld32_async(tbase + i_lo * 64, ra);
+  tmem_wait_ld32(ra);
+  for (int i = i_lo; i < i_hi; ++i) {
+    const float4 *w4 = reinterpret_cast<const float4 *>(wsh + (i - i_lo) * 64);
+    tmem_ld32_async(tbase + i * 64 + 32, rb);            // second half, in flight
+    float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float4 w = w4[k];
+      a0 = ffma2(make_float2(w.x, w.y),
+                 make_float2(fmaxf(ra[4 * k + 0], 0.f), fmaxf(ra[4 * k + 1], 0.f)), a0);
+      a1 = ffma2(make_float2(w.z, w.w),
+                 make_float2(fmaxf(ra[4 * k + 2], 0.f), fmaxf(ra[4 * k + 3], 0.f)), a1);
+    }
+    tmem_wait_ld32(rb);
+    if (i + 1 < i_hi) tmem_ld32_async(tbase + (i + 1) * 64, ra);   // next token, in flight
+    float2 a2 = make_float2(0.f, 0.f), a3 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float4 w = w4[8 + k];
+      a2 = ffma2(make_float2(w.x, w.y),
+                 make_float2(fmaxf(rb[4 * k + 0], 0.f), fmaxf(rb[4 * k + 1], 0.f)), a2);
+      a3 = ffma2(make_float2(w.z, w.w),
+                 make_float2(fmaxf(rb[4 * k + 2], 0.f), fmaxf(rb[4 * k + 3], 0.f)), a3);
+    }
+    store(i, ((a0.x + a0.y) + (a1.x + a1.y)) + ((a2.x + a2.y) + (a3.x + a3.y)));
+    if (i + 1 < i_hi) tmem_wait_ld32(ra);
+  }
+}
+
 __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
 
 // Write the mask bound to row[lo, hi), threads t = 0..nthr-1 of the caller,
@@ -1092,11 +1132,20 @@ __global__ void __launch_bounds__((2 + kEPI + (kFP8 ? 1 : 0) + (kISS - 1)) * 32,
               const int i_lo = kG > 1 ? 0 : min(ntok_s, group * per);
               const int i_hi = kG > 1 ? ntok_s : min(ntok_s, i_lo + per);
               const float *wsh = wrows + (sub * per) * 64;
-              for (int i = i_lo; i < i_hi; ++i) {
-                const float acc = head_sum_h64(tbase + i * 64, wsh + (i - i_lo) * 64);
-                const int lv = qb_last_valid(P, q, i0 + i);
-                if (in_row)
-                  p.scores[q.out0 + (i0 + i) * q.row_len + slot] = slot <= lv ? acc : kMaskBound;
+              if constexpr (kG == 1) {
+                head_sums_h64_pipelined(tbase, i_lo, i_hi, wsh, [&](int i, float acc) {
+                  const int lv = qb_last_valid(P, q, i0 + i);
+                  if (in_row)
+                    p.scores[q.out0 + (i0 + i) * q.row_len + slot] =
+                        slot <= lv ? acc : kMaskBound;
+                });
+              } else {
+                for (int i = i_lo; i < i_hi; ++i) {
+                  const float acc = head_sum_h64(tbase + i * 64, wsh + (i - i_lo) * 64);
+                  const int lv = qb_last_valid(P, q, i0 + i);
+                  if (in_row)
+                    p.scores[q.out0 + (i0 + i) * q.row_len + slot] = slot <= lv ? acc : kMaskBound;
+                }
               }
             } else {
               // any H: walk the sub-block's columns in 16-wide chunks

@@ -319,3 +319,16 @@ def test_paged_unused_table_entries(dsa):
 def test_decode_batch_paged_full_size(dsa):
     wl = syn.WORKLOADS["decode_batch_paged"]
     run_and_check(dsa, wl, syn.generate(wl))
+
+
+def test_causal_with_empty_sequences(dsa):
+    """Zero-length sequences in a packed batch (cu_seqlens repeats a value):
+    the schedule and the top-k's row lookup skip them."""
+    wl = causal_wl((0, 5, 0, 130, 0, 257), H=64, k=64, seed=80)
+    run_and_check(dsa, wl, syn.generate(wl))
+
+
+def test_paged_single_large_page(dsa):
+    """One page holds the whole cache (pages of 4096 slots, S = 3000)."""
+    wl = paged_wl(T=3, H=64, S=3000, k=100, page=4096, seed=81)
+    run_and_check(dsa, wl, syn.generate(wl))

@@ -225,13 +225,16 @@ int main() {
 """
 
 
-def test_invariant_division_of_the_compressed_rule(tmp_path):
+def test_invariant_division_of_the_compressed_rule():
     """The kernels' multiply-and-shift division by compress_ratio equals
     integer division for 31-bit numerators (host build of the same header)."""
+    import pathlib
     import subprocess
-    src = tmp_path / "div_check.cpp"
+    out_dir = pathlib.Path(__file__).resolve().parent.parent / "_build" / "div_check"
+    out_dir.mkdir(parents=True, exist_ok=True)          # _build/ is not versioned
+    src = out_dir / "div_check.cpp"
     src.write_text(_DIV_CHECK)
-    exe = tmp_path / "div_check"
+    exe = out_dir / "div_check"
     subprocess.run(["g++", "-O2", "-std=c++17", "-I", os.path.dirname(ROW_RULE), str(src),
                     "-o", str(exe)], check=True)
     out = subprocess.run([str(exe)], capture_output=True, text=True)

@@ -49,8 +49,14 @@
  *    returns DSA_ERR_INVALID_ARG / DSA_ERR_UNSUPPORTED / DSA_ERR_WORKSPACE and
  *    launches nothing. A failed launch returns DSA_ERR_CUDA.
  *  - Kernels never trap. A device-side wait that runs past its time limit
- *    (4 s) makes the kernel stop, record DSA_ERR_TIMEOUT in the workspace
- *    and exit cleanly; read it with dsa_indexer_get_error.
+ *    (desc->wait_limit_ns, default 4 s) makes the kernel stop, record
+ *    DSA_ERR_TIMEOUT in the workspace and exit cleanly after the copies and
+ *    MMAs it has in flight have landed (those drains have a bound of their
+ *    own, 4 s, whatever the wait limit); read it with dsa_indexer_get_error.
+ *  - CAUSAL: cu_seqlens is checked on the device before any score or top-k
+ *    is written (cu[0] = 0, non-decreasing, cu[num_seqs] = T). A bad array
+ *    makes the kernels of that call write nothing and records
+ *    DSA_ERR_INVALID_ARG in the workspace (dsa_indexer_get_error).
  *  - A workspace belongs to one in-flight call at a time: two calls on
  *    different streams must not share one.
  */
@@ -137,7 +143,31 @@ typedef struct {
                               that hold a valid slot must lie in
                               [0, num_pages); other entries are never used for
                               a score (a page id outside the pool reads as 0)  */
+  uint32_t flags;          /* DSA_FLAG_* bits, 0 for none                       */
+  uint64_t wait_limit_ns;  /* time limit of any single device-side wait; 0 =
+                              the default, 4 s. A wait that runs past it stops
+                              the kernel with DSA_ERR_TIMEOUT (see
+                              dsa_indexer_get_error)                            */
+  const int32_t *cu_seqlens_host; /* CAUSAL with DSA_FLAG_SCORES_IN_WORKSPACE:
+                              a HOST copy of cu_seqlens [num_seqs + 1], read by
+                              dsa_indexer_workspace_size to size the score rows
+                              (the kernels still read the device array). May be
+                              NULL otherwise                                   */
 } dsa_indexer_desc_t;
+
+/* flags */
+/* Top-k only: dsa_indexer_workspace_size adds room for every score row
+ * (after the 256-byte header), and dsa_indexer_forward accepts scores = NULL,
+ * keeping the rows in the workspace, where they are overwritten by the next
+ * call. The index set is the product; the scores are the consumer's optional
+ * by-product (DeepSeek-V3.2 Sparse Indexer Kernel API Reference, Returns). */
+#define DSA_FLAG_SCORES_IN_WORKSPACE 1u
+/* Self-test of the failure path: the score kernel's MMA warp first waits on a
+ * barrier that nothing completes. The wait runs out after wait_limit_ns, the
+ * kernel records DSA_ERR_TIMEOUT, lets its in-flight copies land and exits
+ * with no output written past that point; dsa_indexer_get_error then reports
+ * the timeout. For tests of a caller's error handling: nothing faults. */
+#define DSA_FLAG_SELFTEST_STALL 2u
 
 /*
  * Layouts (all row-major, innermost index last, no padding):
@@ -162,11 +192,13 @@ typedef struct {
  * Scores must hold no NaN when passed to dsa_indexer_topk.
  */
 
-/* Bytes of workspace every call needs (host only; no device work). The
- * workspace is device memory, 256-byte aligned and owned by the caller. It
- * must be zero-filled once before its first use (e.g. cudaMemsetAsync); each
- * call leaves it ready for the next, so it is reused freely between calls
- * that are ordered on the GPU (one stream). */
+/* Bytes of workspace every call needs (host only; no device work): a
+ * 256-byte header, plus, with DSA_FLAG_SCORES_IN_WORKSPACE, the score rows
+ * (4 * T * S bytes; CAUSAL: 4 * sum_i L_i^2 from cu_seqlens_host, which must
+ * then be given). The workspace is device memory, 256-byte aligned and owned
+ * by the caller. It must be zero-filled once before its first use (e.g.
+ * cudaMemsetAsync); each call leaves it ready for the next, so it is reused
+ * freely between calls that are ordered on the GPU (one stream). */
 dsa_status_t dsa_indexer_workspace_size(const dsa_indexer_desc_t *desc,
                                         size_t *bytes);
 
@@ -189,7 +221,11 @@ dsa_status_t dsa_indexer_topk(const dsa_indexer_desc_t *desc,
                               int32_t *topk, void *workspace,
                               size_t workspace_bytes, dsa_stream_t stream);
 
-/* dsa_indexer_score followed by dsa_indexer_topk on the same stream. */
+/* dsa_indexer_score followed by dsa_indexer_topk on the same stream.
+ * scores = NULL (top-k only) needs DSA_FLAG_SCORES_IN_WORKSPACE and a
+ * workspace of the size dsa_indexer_workspace_size reports for it; the rows
+ * then live in the workspace (DSA_ERR_WORKSPACE when it is too small,
+ * DSA_ERR_INVALID_ARG without the flag). */
 dsa_status_t dsa_indexer_forward(const dsa_indexer_desc_t *desc,
                                  const void *q, const uint8_t *q_scale,
                                  const float *w, const void *k,
@@ -207,7 +243,8 @@ dsa_status_t dsa_indexer_forward(const dsa_indexer_desc_t *desc,
  * the library, held by every GPU that loads it until the process exits; a
  * problem whose workspace size exceeds it returns DSA_ERR_WORKSPACE. The
  * first call on a device looks up that array's address (do it before any
- * stream capture). Every call clears the scratch on `stream`; all calls share
+ * stream capture); the address is kept for the life of the process, so a
+ * cudaDeviceReset after that first call is not supported. Every call clears the scratch on `stream`; all calls share
  * it, so calls that overlap on the GPU race and must be serialised by the
  * caller. Device-side timeouts are not reported by this entry point. */
 dsa_status_t dsa_indexer_forward_noalloc(const dsa_indexer_desc_t *desc,

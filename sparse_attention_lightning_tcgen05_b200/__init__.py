@@ -29,6 +29,8 @@ DSA_MASK_POSITIONS = 0
 DSA_MASK_CAUSAL = 1
 DSA_MASK_COMPRESSED = 2
 DSA_MASK_BOUND = float.fromhex("-0x1.FEp127")
+DSA_FLAG_SCORES_IN_WORKSPACE = 1
+DSA_FLAG_SELFTEST_STALL = 2
 
 # Every symbol include/dsa_indexer.h declares.
 EXPORTS = ("dsa_indexer_workspace_size", "dsa_indexer_score", "dsa_indexer_topk",
@@ -44,7 +46,9 @@ class dsa_indexer_desc_t(ctypes.Structure):
                 ("dtype", ctypes.c_int), ("mask", ctypes.c_int),
                 ("query_start", ctypes.c_int64), ("compress_ratio", ctypes.c_int32),
                 ("page_size", ctypes.c_int32), ("pages_per_seq", ctypes.c_int32),
-                ("num_pages", ctypes.c_int32), ("block_table", ctypes.c_void_p)]
+                ("num_pages", ctypes.c_int32), ("block_table", ctypes.c_void_p),
+                ("flags", ctypes.c_uint32), ("wait_limit_ns", ctypes.c_uint64),
+                ("cu_seqlens_host", ctypes.c_void_p)]
 
 
 class DsaError(RuntimeError):
@@ -87,14 +91,22 @@ def _ptr(x) -> int | None:
 def make_desc(T, H, index_topk, *, D=128, S=0, k_seq_stride=0, num_seqs=0,
               cu_seqlens=None, dtype=DSA_KV_BF16, mask=DSA_MASK_POSITIONS,
               query_start=0, compress_ratio=0, page_size=0, pages_per_seq=0,
-              num_pages=0, block_table=None):
+              num_pages=0, block_table=None, flags=0, wait_limit_ns=0,
+              cu_seqlens_host=None):
+    """A descriptor. cu_seqlens_host: a contiguous int32 numpy array (host
+    memory) that the caller keeps alive while the descriptor is used."""
+    host_cu = None
+    if cu_seqlens_host is not None:
+        assert cu_seqlens_host.dtype.name == "int32" and cu_seqlens_host.flags.c_contiguous
+        host_cu = cu_seqlens_host.ctypes.data
     return dsa_indexer_desc_t(T=T, H=H, D=D, index_topk=index_topk, S=S,
                               k_seq_stride=k_seq_stride, num_seqs=num_seqs,
                               cu_seqlens=_ptr(cu_seqlens), dtype=dtype,
                               mask=mask, query_start=query_start,
                               compress_ratio=compress_ratio, page_size=page_size,
                               pages_per_seq=pages_per_seq, num_pages=num_pages,
-                              block_table=_ptr(block_table))
+                              block_table=_ptr(block_table), flags=flags,
+                              wait_limit_ns=wait_limit_ns, cu_seqlens_host=host_cu)
 
 
 def dsa_status_string(status: int) -> str:

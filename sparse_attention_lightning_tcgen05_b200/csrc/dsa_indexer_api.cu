@@ -13,6 +13,7 @@
 
 #include "dsa_indexer.h"
 #include "dsa_launch.h"
+#include "cu_check.cuh"
 #include "score_kernel.cuh"
 #include "topk_cluster.cuh"
 #include "topk_rows.cuh"
@@ -24,16 +25,20 @@ using dsa::ScoreParams;
 using dsa::ScoreSmem;
 using dsa::TopkParams;
 
-constexpr uint64_t kWaitLimitNs = 4000000000ull;   // 4 s for any single wait
+constexpr uint64_t kWaitLimitNs = 4000000000ull;   // default limit of any single wait
+constexpr uint64_t kDrainLimitNs = 4000000000ull;  // drains of in-flight copies / MMAs
 constexpr int kMaxDevices = 64;
 constexpr uint32_t kMaxSmemPerBlock = 232448;      // 227 KB opt-in limit of sm_100
 
 // Words of the workspace header.
 // err/err_info: first device-side failure since the last get_error (sticky).
+// cu_bad: written by the cu_seqlens check of every CAUSAL call, read by that
+// call's score and top-k kernels.
 struct WsHeader {
   unsigned int err;
   unsigned int err_info;
-  unsigned int reserved[62];
+  unsigned int cu_bad;
+  unsigned int reserved[61];
 };
 static_assert(sizeof(WsHeader) == kWorkspaceHeader, "header size");
 
@@ -98,6 +103,8 @@ bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 dsa_status_t check_desc(const dsa_indexer_desc_t *d) {
   if (!d) return DSA_ERR_INVALID_ARG;
   if (d->T < 1 || d->H < 1 || d->index_topk < 1) return DSA_ERR_INVALID_ARG;
+  if (d->flags & ~(DSA_FLAG_SCORES_IN_WORKSPACE | DSA_FLAG_SELFTEST_STALL))
+    return DSA_ERR_INVALID_ARG;
   if (d->dtype != DSA_KV_BF16 && d->dtype != DSA_KV_FP8_E4M3_E8M0_B32) return DSA_ERR_INVALID_ARG;
   if (d->mask != DSA_MASK_POSITIONS && d->mask != DSA_MASK_CAUSAL &&
       d->mask != DSA_MASK_COMPRESSED)
@@ -150,6 +157,36 @@ dsa_status_t check_workspace(const void *ws, size_t bytes) {
   if (!ws || !aligned(ws, 256) || bytes < kWorkspaceHeader) return DSA_ERR_WORKSPACE;
   return DSA_OK;
 }
+
+// Floats of all score rows (host): T*S, or for CAUSAL sum_i L_i^2 from the
+// host copy of cu_seqlens, which is checked like the device array is.
+dsa_status_t score_elems(const dsa_indexer_desc_t *d, int64_t *n) {
+  if (d->mask != DSA_MASK_CAUSAL) {
+    *n = static_cast<int64_t>(d->T) * d->S;
+    return DSA_OK;
+  }
+  const int32_t *cu = d->cu_seqlens_host;
+  if (!cu || cu[0] != 0 || cu[d->num_seqs] != d->T) return DSA_ERR_INVALID_ARG;
+  int64_t total = 0;
+  for (int i = 0; i < d->num_seqs; ++i) {
+    if (cu[i + 1] < cu[i]) return DSA_ERR_INVALID_ARG;
+    const int64_t L = cu[i + 1] - cu[i];
+    total += L * L;
+  }
+  *n = total;
+  return DSA_OK;
+}
+
+// The score rows of a top-k-only call: right after the workspace header.
+// Returns the floats the workspace holds for them (-1 when the caller's
+// buffer is used and its size is unknown).
+int64_t workspace_scores(void *ws, size_t ws_bytes, float **scores) {
+  if (*scores != nullptr) return -1;
+  *scores = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + kWorkspaceHeader);
+  return static_cast<int64_t>((ws_bytes - kWorkspaceHeader) / 4);
+}
+
+
 
 // ---- tensor maps -------------------------------------------------------------------------
 
@@ -283,13 +320,29 @@ ScoreLaunch choose_score(const dsa_indexer_desc_t *d) {
                               1, 1, tq, round16(tq * H), 128, true};
 }
 
+// CAUSAL: check cu_seqlens on the device (one CTA) before the kernels that
+// read it; they skip their work when it fails. cap_elems >= 0 also bounds the
+// score rows (they live in a workspace of that many floats).
+dsa_status_t launch_cu_check(const dsa_indexer_desc_t *d, WsHeader *ws, int64_t cap_elems,
+                             cudaStream_t stream) {
+  if (launch_pdl(dsa::cu_seqlens_check_kernel<256>, 1, 256, 0, stream, 0, d->cu_seqlens,
+                 d->num_seqs, d->T, static_cast<long long>(cap_elems), &ws->cu_bad,
+                 &ws->err) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  return DSA_OK;
+}
+
 dsa_status_t launch_score(const dsa_indexer_desc_t *d, const void *q, const uint8_t *q_scale,
                           const float *w, const void *k, const uint8_t *k_scale,
                           const int32_t *positions, float *scores, WsHeader *ws,
-                          cudaStream_t stream) {
+                          int64_t cap_elems, cudaStream_t stream) {
   DeviceInfo *dev = nullptr;
   dsa_status_t st = device_info(&dev);
   if (st != DSA_OK) return st;
+  if (d->mask == DSA_MASK_CAUSAL) {
+    st = launch_cu_check(d, ws, cap_elems, stream);
+    if (st != DSA_OK) return st;
+  }
   const ScoreLaunch L = choose_score(d);
   const ScoreSmem plan(L.stages, L.qbuf, L.nsub, L.n_cols, L.fp8, L.epi, L.tiles);
   // the attribute is set once per kernel: use the widest query block it runs
@@ -376,7 +429,10 @@ dsa_status_t launch_score(const dsa_indexer_desc_t *d, const void *q, const uint
   p.n_cols = L.n_cols;
   p.err = &ws->err;
   p.err_info = &ws->err_info;
-  p.wait_limit_ns = kWaitLimitNs;
+  p.cu_bad = &ws->cu_bad;
+  p.wait_limit_ns = d->wait_limit_ns ? d->wait_limit_ns : kWaitLimitNs;
+  p.drain_limit_ns = kDrainLimitNs;
+  p.selftest_stall = (d->flags & DSA_FLAG_SELFTEST_STALL) ? 1 : 0;
   // With one query buffer the next block's query cannot load while the
   // current block's MMAs run: a block start costs about 3/4 of a key tile
   // (measured on an 8192-token prefill), so the split between CTAs counts
@@ -409,11 +465,18 @@ dsa_status_t launch_topk_rows(DeviceInfo *dev, int which, int T, const TopkParam
 }
 
 dsa_status_t launch_topk(const dsa_indexer_desc_t *d, const float *scores,
-                         const int32_t *positions, int32_t *topk, cudaStream_t stream) {
+                         const int32_t *positions, int32_t *topk, WsHeader *ws, bool check_cu,
+                         int64_t cap_elems, cudaStream_t stream) {
   DeviceInfo *dev = nullptr;
   dsa_status_t st = device_info(&dev);
   if (st != DSA_OK) return st;
+  if (check_cu && d->mask == DSA_MASK_CAUSAL) {
+    st = launch_cu_check(d, ws, cap_elems, stream);
+    if (st != DSA_OK) return st;
+  }
   TopkParams p{};
+  p.cu_bad = &ws->cu_bad;
+  p.err = &ws->err;
   p.mode = d->mask == DSA_MASK_CAUSAL ? dsa::kModeCausal : dsa::kModePositions;
   p.T = d->T;
   p.S = d->S;
@@ -424,14 +487,17 @@ dsa_status_t launch_topk(const dsa_indexer_desc_t *d, const float *scores,
   p.scores = scores;
   p.topk = topk;
   p.k = d->index_topk;
-  // Decode-style rows of at most 4096 slots (pooled keys, short caches): one
-  // CTA a row, the row held in registers. Longer decode rows are few and
-  // long: a cluster of C CTAs per row (up to 8, about 4096 slots each), the
-  // row staged across their shared memories. Prefill rows are many: 512
-  // threads a row and a smaller stage, so that several rows run on each SM.
-  if (p.mode == dsa::kModePositions && d->S <= 4096) {
-    const dsa_status_t rs = d->S <= 2048 ? launch_topk_rows<256, 8>(dev, 0, d->T, p, stream)
-                                         : launch_topk_rows<256, 16>(dev, 1, d->T, p, stream);
+  // Decode-style rows of at most 4093 slots (pooled keys, short caches): one
+  // CTA a row, the row held in registers. A row's buffer starts at the
+  // 16-byte boundary at or before it, up to 3 floats early, so an instance
+  // holding NT*KPT floats takes rows of up to NT*KPT - 3 slots. Longer decode
+  // rows are few and long: a cluster of C CTAs per row (up to 8, about 4096
+  // slots each), the row staged across their shared memories. Prefill rows
+  // are many: 512 threads a row and a smaller stage, so that several rows run
+  // on each SM.
+  if (p.mode == dsa::kModePositions && d->S + 3 <= 4096) {
+    const dsa_status_t rs = d->S + 3 <= 2048 ? launch_topk_rows<256, 8>(dev, 0, d->T, p, stream)
+                                             : launch_topk_rows<256, 16>(dev, 1, d->T, p, stream);
     if (rs != DSA_OK) return rs;
     return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
   }
@@ -480,9 +546,16 @@ extern "C" {
 
 dsa_status_t dsa_indexer_workspace_size(const dsa_indexer_desc_t *desc, size_t *bytes) {
   if (!bytes) return DSA_ERR_INVALID_ARG;
-  const dsa_status_t st = check_desc(desc);
+  dsa_status_t st = check_desc(desc);
   if (st != DSA_OK) return st;
-  *bytes = kWorkspaceHeader;
+  size_t n = kWorkspaceHeader;
+  if (desc->flags & DSA_FLAG_SCORES_IN_WORKSPACE) {
+    int64_t elems = 0;
+    st = score_elems(desc, &elems);
+    if (st != DSA_OK) return st;
+    n += static_cast<size_t>(elems) * 4;
+  }
+  *bytes = n;
   return DSA_OK;
 }
 
@@ -497,7 +570,7 @@ dsa_status_t dsa_indexer_score(const dsa_indexer_desc_t *desc, const void *q,
   if (st != DSA_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   return launch_score(desc, q, q_scale, w, k, k_scale, positions, scores,
-                      static_cast<WsHeader *>(workspace), s);
+                      static_cast<WsHeader *>(workspace), -1, s);
 }
 
 dsa_status_t dsa_indexer_topk(const dsa_indexer_desc_t *desc, const float *scores,
@@ -511,7 +584,8 @@ dsa_status_t dsa_indexer_topk(const dsa_indexer_desc_t *desc, const float *score
   st = check_workspace(workspace, workspace_bytes);
   if (st != DSA_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  return launch_topk(desc, scores, positions, topk, s);
+  return launch_topk(desc, scores, positions, topk, static_cast<WsHeader *>(workspace), true,
+                     -1, s);
 }
 
 dsa_status_t dsa_indexer_forward(const dsa_indexer_desc_t *desc, const void *q,
@@ -520,15 +594,27 @@ dsa_status_t dsa_indexer_forward(const dsa_indexer_desc_t *desc, const void *q,
                                  float *scores, int32_t *topk, void *workspace,
                                  size_t workspace_bytes, dsa_stream_t stream) {
   dsa_status_t st = check_desc(desc);
-  if (st == DSA_OK) st = check_inputs(desc, q, q_scale, w, k, k_scale, positions, scores);
+  if (st != DSA_OK) return st;
+  st = check_workspace(workspace, workspace_bytes);
+  if (st != DSA_OK) return st;
+  // top-k only: the score rows go to the workspace, which must hold them
+  int64_t cap = -1;
+  if (!scores) {
+    if (!(desc->flags & DSA_FLAG_SCORES_IN_WORKSPACE)) return DSA_ERR_INVALID_ARG;
+    int64_t elems = 0;
+    st = score_elems(desc, &elems);
+    if (st != DSA_OK) return st;
+    cap = workspace_scores(workspace, workspace_bytes, &scores);
+    if (cap < elems) return DSA_ERR_WORKSPACE;
+  }
+  st = check_inputs(desc, q, q_scale, w, k, k_scale, positions, scores);
   if (st == DSA_OK && (!topk || !aligned(topk, 4))) st = DSA_ERR_INVALID_ARG;
-  if (st == DSA_OK) st = check_workspace(workspace, workspace_bytes);
   if (st != DSA_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  st = launch_score(desc, q, q_scale, w, k, k_scale, positions, scores,
-                    static_cast<WsHeader *>(workspace), s);
+  WsHeader *ws = static_cast<WsHeader *>(workspace);
+  st = launch_score(desc, q, q_scale, w, k, k_scale, positions, scores, ws, cap, s);
   if (st != DSA_OK) return st;
-  return launch_topk(desc, scores, positions, topk, s);
+  return launch_topk(desc, scores, positions, topk, ws, false, cap, s);
 }
 
 dsa_status_t dsa_indexer_get_error(const void *workspace, dsa_stream_t stream,

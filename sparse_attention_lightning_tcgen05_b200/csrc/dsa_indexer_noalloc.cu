@@ -14,7 +14,9 @@
 // GPU that loads the library holds it until the process exits. Host code never
 // uses its name as an address; the device address is looked up once per
 // device with cudaGetSymbolAddress, on the first call made with that device
-// current, so that first call should come before any stream capture. All calls
+// current, so that first call should come before any stream capture. The
+// address is kept for the life of the process: a cudaDeviceReset after the
+// first call (which unloads the library's module) is not supported. All calls
 // share the array: calls that overlap on the GPU (different streams, or
 // different host threads on one device) race on it and must be serialised by
 // the caller. Each call clears the scratch on its stream before the kernels
@@ -75,8 +77,8 @@ extern "C" dsa_status_t dsa_indexer_forward_noalloc(
   if (st != DSA_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(scratch, 0, need, s) != cudaSuccess) return DSA_ERR_CUDA;
-  st = dsa_host::launch_score(desc, q, q_scale, w, k, k_scale, positions, scores,
-                              static_cast<dsa_host::WsHeader *>(scratch), s);
+  dsa_host::WsHeader *ws = static_cast<dsa_host::WsHeader *>(scratch);
+  st = dsa_host::launch_score(desc, q, q_scale, w, k, k_scale, positions, scores, ws, -1, s);
   if (st != DSA_OK) return st;
-  return dsa_host::launch_topk(desc, scores, positions, topk, s);
+  return dsa_host::launch_topk(desc, scores, positions, topk, ws, false, -1, s);
 }

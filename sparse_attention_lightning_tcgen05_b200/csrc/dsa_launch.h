@@ -20,11 +20,16 @@ dsa_status_t check_desc(const dsa_indexer_desc_t *d);
 dsa_status_t check_inputs(const dsa_indexer_desc_t *d, const void *q, const uint8_t *q_scale,
                           const float *w, const void *k, const uint8_t *k_scale,
                           const int32_t *positions, const float *scores);
+// cap_elems: floats the score buffer is known to hold (a top-k-only call's
+// workspace), or -1 when the caller's buffer is used. launch_score runs the
+// CAUSAL cu_seqlens check first; launch_topk runs it when check_cu is set
+// (a top-k call of its own).
 dsa_status_t launch_score(const dsa_indexer_desc_t *d, const void *q, const uint8_t *q_scale,
                           const float *w, const void *k, const uint8_t *k_scale,
                           const int32_t *positions, float *scores, WsHeader *ws,
-                          cudaStream_t stream);
+                          int64_t cap_elems, cudaStream_t stream);
 dsa_status_t launch_topk(const dsa_indexer_desc_t *d, const float *scores,
-                         const int32_t *positions, int32_t *topk, cudaStream_t stream);
+                         const int32_t *positions, int32_t *topk, WsHeader *ws, bool check_cu,
+                         int64_t cap_elems, cudaStream_t stream);
 
 }  // namespace dsa_host

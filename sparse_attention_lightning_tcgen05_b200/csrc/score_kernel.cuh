@@ -71,7 +71,10 @@ struct ScoreParams {
   int n_cols;                // MMA N per sub-block: round_up(tq_sub*H, 16)
   unsigned int *err;
   unsigned int *err_info;
-  uint64_t wait_limit_ns;
+  const unsigned int *cu_bad;   // CAUSAL: set by the cu_seqlens check -> no work
+  uint64_t wait_limit_ns;       // any single wait
+  uint64_t drain_limit_ns;      // the drains on the way out (not the wait limit)
+  int selftest_stall;           // the MMA warp first waits on a barrier nothing completes
 };
 
 __host__ __device__ constexpr int sf_atoms(int n_cols) { return (n_cols + 127) / 128; }
@@ -710,7 +713,7 @@ __global__ void __launch_bounds__((2 + kEPI + (kFP8 ? 1 : 0) + (kISS - 1)) * 32,
   static_assert(kISS == 1 || kISS == 2, "issuers");
   constexpr int kSFWarp = 2 + kEPI;                        // fp8 scale-factor warp
   constexpr int kIss2Warp = 2 + kEPI + (kFP8 ? 1 : 0);     // second MMA issuer
-  static_assert(3 * (kSTAGES + kQBUF) + 2 * kNACC <= 64, "barrier budget");
+  static_assert(3 * (kSTAGES + kQBUF) + 2 * kNACC <= 63, "barrier budget");
   constexpr int kGroups = kEPI / 4;
   constexpr int kAPS = kG;                       // accumulators per slot
   extern __shared__ uint8_t smem_raw[];
@@ -730,6 +733,7 @@ __global__ void __launch_bounds__((2 + kEPI + (kFP8 ? 1 : 0) + (kISS - 1)) * 32,
   uint64_t *acc_empty = acc_full + kNACC;        // [kNACC]
   uint64_t *sf_ready = acc_empty + kNACC;        // [kSTAGES] fp8: A scales in TMEM
   uint64_t *sfq_ready = sf_ready + kSTAGES;      // [kQBUF]   fp8: B scales in TMEM
+  uint64_t *stall_bar = bars + 63;               // self-test: never completed
   uint32_t *misc = reinterpret_cast<uint32_t *>(smem + L.off_misc);
   uint32_t *tmem_base_slot = misc;               // written by tcgen05.alloc
   volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 1);
@@ -755,6 +759,7 @@ __global__ void __launch_bounds__((2 + kEPI + (kFP8 ? 1 : 0) + (kISS - 1)) * 32,
       for (int i = 0; i < kSTAGES; ++i) mbar_init(sf_ready + i, 1);
       for (int i = 0; i < kQBUF; ++i) mbar_init(sfq_ready + i, 1);
     }
+    mbar_init(stall_bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmap_k);
@@ -783,7 +788,12 @@ __global__ void __launch_bounds__((2 + kEPI + (kFP8 ? 1 : 0) + (kISS - 1)) * 32,
   if (pos_staged) P.positions = spos;
   if (warp == 0) {
     CtaRange R;
-    cta_range(P, tqt, R);
+    // CAUSAL: a cu_seqlens array that failed its check leaves the CTA no work
+    if (kMODE == kModeCausal && *p.cu_bad) {
+      R = CtaRange{};
+    } else {
+      cta_range(P, tqt, R);
+    }
     if (lane == 0) *range_slot = R;
   }
   tc_fence_before_sync();
@@ -868,14 +878,16 @@ __global__ void __launch_bounds__((2 + kEPI + (kFP8 ? 1 : 0) + (kISS - 1)) * 32,
       }
       // Let every copy this thread started land before the CTA can exit.
       for (int i = 0; i < kSTAGES; ++i)
-        if (k_issued >> i & 1u) mbar_drain(full_k + i, k_last_phase >> i & 1u, p.wait_limit_ns);
+        if (k_issued >> i & 1u) mbar_drain(full_k + i, k_last_phase >> i & 1u, p.drain_limit_ns);
       for (int i = 0; i < kQBUF; ++i)
-        if (q_issued >> i & 1u) mbar_drain(q_full + i, q_last_phase >> i & 1u, p.wait_limit_ns);
+        if (q_issued >> i & 1u) mbar_drain(q_full + i, q_last_phase >> i & 1u, p.drain_limit_ns);
     }
   } else if (warp == 1 || (kISS == 2 && warp == kIss2Warp)) {
     // ---------------- MMA issuers (each walks every item, issues its own) ----
     const int my_parity = warp == 1 ? 0 : 1;
-    if (R.a_count > 0) {
+    // self-test of the failure path: a wait that runs out (nothing arrives)
+    const bool stalled = p.selftest_stall && warp == 1 && !mbar_wait(stall_bar, 0, ctl, 31);
+    if (R.a_count > 0 && !stalled) {
       Ring st, qb, ac;
       uint64_t *last_commit = nullptr;
       uint32_t last_commit_phase = 0;
@@ -967,7 +979,7 @@ __global__ void __launch_bounds__((2 + kEPI + (kFP8 ? 1 : 0) + (kISS - 1)) * 32,
         }
       }
       // MMAs still in flight must finish before TMEM is released.
-      if (lane == 0 && last_commit) mbar_drain(last_commit, last_commit_phase, p.wait_limit_ns);
+      if (lane == 0 && last_commit) mbar_drain(last_commit, last_commit_phase, p.drain_limit_ns);
       __syncwarp();
     }
   } else if (kFP8 && warp == kSFWarp) {
@@ -1040,7 +1052,7 @@ __global__ void __launch_bounds__((2 + kEPI + (kFP8 ? 1 : 0) + (kISS - 1)) * 32,
         }
       }
       // copies still in flight must land before TMEM is released
-      if (lane == 0 && last_commit) mbar_drain(last_commit, last_commit_phase, p.wait_limit_ns);
+      if (lane == 0 && last_commit) mbar_drain(last_commit, last_commit_phase, p.drain_limit_ns);
       __syncwarp();
     }
   } else if (warp < 2 + kEPI) {

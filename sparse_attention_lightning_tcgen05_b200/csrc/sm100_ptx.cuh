@@ -185,8 +185,8 @@ __device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
     }
   }
   *ctl.abort = 1;
-  atomicExch(ctl.err, kStatusTimeout);
-  atomicExch(ctl.err_info, site);
+  // the first failure since the last report is the one kept
+  if (atomicCAS(ctl.err, 0u, kStatusTimeout) == 0u) atomicExch(ctl.err_info, site);
   return false;
 }
 

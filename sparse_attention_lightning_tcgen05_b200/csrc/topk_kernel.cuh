@@ -44,6 +44,8 @@ struct TopkParams {
   int *topk;
   int k;
   int stage_cap;            // keys a CTA may stage in shared memory
+  const unsigned int *cu_bad;   // CAUSAL: set by the cu_seqlens check -> no work
+  unsigned int *err;        // device status word (first failure kept)
 };
 
 template <int NT>
@@ -276,6 +278,8 @@ __global__ void __launch_bounds__(NT) topk_kernel(const TopkParams p) {
   // scores (and positions) come from earlier work on the stream
   grid_dep_wait();
   grid_dep_launch_dependents();
+  // CAUSAL: a cu_seqlens array that failed its check -> write nothing
+  if (p.mode == kModeCausal && *p.cu_bad) return;
 
   const float *row;
   int64_t nvalid;

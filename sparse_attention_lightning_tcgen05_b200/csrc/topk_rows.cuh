@@ -109,6 +109,12 @@ struct RowJob {
   int kind;            // 0: too long for this instance, 1: n <= k (no selection), 2: select
 };
 
+// Floats of a row's buffer that its valid slots occupy: the buffer starts at
+// the 16-byte boundary at or before the row, h = 0..3 floats earlier.
+__device__ __forceinline__ int64_t rows_span(const float *row, int64_t nvalid) {
+  return nvalid + static_cast<int64_t>((reinterpret_cast<uintptr_t>(row) & 15u) / 4u);
+}
+
 template <int NT, int KPT>
 __device__ __forceinline__ RowJob rows_job(const TopkParams &p, int t, int lane) {
   RowJob j;
@@ -116,7 +122,7 @@ __device__ __forceinline__ RowJob rows_job(const TopkParams &p, int t, int lane)
   rows_geometry(p, t, lane, j.row, nvalid);
   j.out = p.topk + static_cast<int64_t>(t) * p.k;
   j.n = static_cast<uint32_t>(nvalid < 0 ? 0 : (nvalid > 0x7fffffff ? 0x7fffffff : nvalid));
-  j.kind = nvalid <= p.k ? 1 : (nvalid > static_cast<int64_t>(NT) * KPT ? 0 : 2);
+  j.kind = nvalid <= p.k ? 1 : (rows_span(j.row, nvalid) > static_cast<int64_t>(NT) * KPT ? 0 : 2);
   return j;
 }
 
@@ -450,7 +456,10 @@ __global__ void __launch_bounds__(NT) topk_rows_kernel(const TopkParams p) {
     for (uint32_t i = tid; i < k; i += NT) job.out[i] = i < job.n ? static_cast<int>(i) : -1;
     return;
   }
-  if (job.kind == 0) return;             // the host sends no row this long
+  if (job.kind == 0) {                   // the host sends no row this long
+    if (tid == 0) atomicCAS(p.err, 0u, 2u);   // DSA_ERR_UNSUPPORTED, never expected
+    return;
+  }
   rows_prefetch<NT, KPT>(job, rows_buf);
   cp_async_commit();
   cp_async_wait<0>();

@@ -9,7 +9,7 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import (DSA_KV_BF16, DSA_MASK_CAUSAL, DSA_MASK_COMPRESSED, DSA_MASK_POSITIONS,
+from . import (DSA_FLAG_SCORES_IN_WORKSPACE, DSA_KV_BF16, DSA_MASK_CAUSAL, DSA_MASK_COMPRESSED, DSA_MASK_POSITIONS,
                dsa_indexer_forward, dsa_indexer_get_error, dsa_indexer_score,
                dsa_indexer_topk, dsa_indexer_workspace_size, make_desc)
 
@@ -31,7 +31,10 @@ class DeviceProblem:
     def __init__(self, *, mode, T, H, index_topk, q, w, k, dtype=DSA_KV_BF16,
                  S=0, k_seq_stride=0, cu_seqlens=None, positions=None,
                  q_scale=None, k_scale=None, query_start=0, compress_ratio=0,
-                 page_size=0, block_table=None, num_pages=0, device="cuda"):
+                 page_size=0, block_table=None, num_pages=0, device="cuda",
+                 topk_only=False, wait_limit_ns=0):
+        """topk_only: scores stay in the workspace (DSA_FLAG_SCORES_IN_WORKSPACE,
+        forward with scores = NULL); self.scores is then a view of them."""
         self.mode, self.T, self.H, self.k = mode, T, H, index_topk
         self.S, self.dtype = S, dtype
         self.q = _dev(q, device)
@@ -42,29 +45,39 @@ class DeviceProblem:
         self.positions = _dev(positions, device)
         self.cu_seqlens = _dev(cu_seqlens, device)
         self.block_table = _dev(block_table, device)
+        self._cu_host = None
         if mode == DSA_MASK_CAUSAL:
             cu = np.asarray(cu_seqlens if not isinstance(cu_seqlens, torch.Tensor)
                             else cu_seqlens.cpu().numpy(), np.int64)
             lens = np.diff(cu)
             self.num_seqs = len(lens)
             n_scores = int((lens * lens).sum())
+            self._cu_host = np.ascontiguousarray(cu, np.int32)
         else:
             self.num_seqs = 0
             n_scores = T * S
+        self.topk_only = topk_only
         self.desc = make_desc(T, H, index_topk, S=S, k_seq_stride=k_seq_stride,
                               num_seqs=self.num_seqs, cu_seqlens=self.cu_seqlens,
                               dtype=dtype, mask=mode, query_start=query_start,
                               compress_ratio=compress_ratio, page_size=page_size,
                               pages_per_seq=(0 if block_table is None
                                              else int(block_table.shape[1])),
-                              num_pages=num_pages, block_table=self.block_table)
-        self.scores = torch.empty(n_scores, dtype=torch.float32, device=device)
+                              num_pages=num_pages, block_table=self.block_table,
+                              flags=DSA_FLAG_SCORES_IN_WORKSPACE if topk_only else 0,
+                              wait_limit_ns=wait_limit_ns,
+                              cu_seqlens_host=self._cu_host)
         self.topk = torch.empty((T, index_topk), dtype=torch.int32, device=device)
         self.ws_bytes = dsa_indexer_workspace_size(self.desc)
         self.workspace = torch.zeros(self.ws_bytes, dtype=torch.uint8, device=device)
+        if topk_only:
+            # the rows the library keeps in the workspace, after its header
+            self.scores = self.workspace[256:256 + 4 * n_scores].view(torch.float32)
+        else:
+            self.scores = torch.empty(n_scores, dtype=torch.float32, device=device)
 
     @classmethod
-    def from_workload(cls, wl, inputs, device="cuda"):
+    def from_workload(cls, wl, inputs, device="cuda", **kw):
         """From a dsa_synth.Workload and its generated inputs."""
         mode = {0: DSA_MASK_POSITIONS, 1: DSA_MASK_CAUSAL,
                 2: DSA_MASK_COMPRESSED}[wl.mode]
@@ -77,7 +90,7 @@ class DeviceProblem:
                    query_start=wl.query_start, compress_ratio=wl.compress_ratio,
                    page_size=wl.page_size if wl.paged else 0,
                    block_table=inputs.get("block_table"), num_pages=wl.num_pages,
-                   device=device)
+                   device=device, **kw)
 
     def _stream(self, stream):
         if stream is None:
@@ -96,8 +109,8 @@ class DeviceProblem:
     def forward(self, stream=None):
         dsa_indexer_forward(self.desc, self.q, self.q_scale, self.w,
                             self.k_cache, self.k_scale, self.positions,
-                            self.scores, self.topk, self.workspace,
-                            self.ws_bytes, self._stream(stream))
+                            None if self.topk_only else self.scores, self.topk,
+                            self.workspace, self.ws_bytes, self._stream(stream))
 
     def device_status(self, stream=None) -> int:
         return dsa_indexer_get_error(self.workspace, self._stream(stream))

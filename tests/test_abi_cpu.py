@@ -240,3 +240,89 @@ def test_invariant_division_of_the_compressed_rule():
     out = subprocess.run([str(exe)], capture_output=True, text=True)
     bad, n = map(int, out.stdout.split())
     assert out.returncode == 0 and bad == 0 and n > 10**6
+
+
+_LAYOUT = r"""
+#include <stddef.h>
+#include <stdio.h>
+#include "dsa_indexer.h"
+#define F(m) printf(#m " %zu\n", offsetof(dsa_indexer_desc_t, m))
+int main(void) {
+  F(T); F(H); F(D); F(index_topk); F(S); F(k_seq_stride); F(num_seqs);
+  F(cu_seqlens); F(dtype); F(mask); F(query_start); F(compress_ratio);
+  F(page_size); F(pages_per_seq); F(num_pages); F(block_table); F(flags);
+  F(wait_limit_ns); F(cu_seqlens_host);
+  printf("sizeof %zu\n", sizeof(dsa_indexer_desc_t));
+  return 0;
+}
+"""
+
+
+def test_descriptor_layout_matches_the_c_header():
+    """Every field of the binding's descriptor sits where a C compiler puts
+    it (host build of the header; gcc)."""
+    import pathlib
+    import subprocess
+    out_dir = pathlib.Path(__file__).resolve().parent.parent / "_build" / "layout"
+    out_dir.mkdir(parents=True, exist_ok=True)
+    src = out_dir / "layout.c"
+    src.write_text(_LAYOUT)
+    exe = out_dir / "layout"
+    subprocess.run(["gcc", "-O0", "-I", os.path.dirname(HEADER), str(src), "-o", str(exe)],
+                   check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout
+    got = dict(line.split() for line in out.strip().splitlines())
+    f = dsa.dsa_indexer_desc_t
+    for name, off in got.items():
+        want = ctypes.sizeof(f) if name == "sizeof" else getattr(f, name).offset
+        assert int(off) == want, name
+
+
+def test_workspace_size_of_a_topk_only_call():
+    """With DSA_FLAG_SCORES_IN_WORKSPACE the workspace also holds every score
+    row after its 256-byte header: 4*T*S bytes, or 4*sum L_i^2 for packed
+    causal rows (from the host copy of cu_seqlens)."""
+    import numpy as np
+    F = dsa.DSA_FLAG_SCORES_IN_WORKSPACE
+    assert dsa.dsa_indexer_workspace_size(good_desc(flags=F)) == 256 + 4 * 4 * 1024
+    assert dsa.dsa_indexer_workspace_size(compressed_desc(flags=F)) == 256 + 4 * 64 * 300
+    cu = np.array([0, 3, 3, 10, 17], np.int32)
+    d = dsa.make_desc(17, 64, 16, mask=dsa.DSA_MASK_CAUSAL, num_seqs=4, cu_seqlens=1 << 20,
+                      flags=F, cu_seqlens_host=cu)
+    assert dsa.dsa_indexer_workspace_size(d) == 256 + 4 * (9 + 0 + 49 + 49)
+    d.flags = 0
+    assert dsa.dsa_indexer_workspace_size(d) == 256
+    for bad in ([1, 3, 3, 10, 17], [0, 3, 2, 10, 17], [0, 3, 3, 10, 16]):
+        arr = np.array(bad, np.int32)
+        d = dsa.make_desc(17, 64, 16, mask=dsa.DSA_MASK_CAUSAL, num_seqs=4,
+                          cu_seqlens=1 << 20, flags=F, cu_seqlens_host=arr)
+        with pytest.raises(dsa.DsaError) as e:
+            dsa.dsa_indexer_workspace_size(d)
+        assert e.value.status == dsa.DSA_ERR_INVALID_ARG
+    d = dsa.make_desc(17, 64, 16, mask=dsa.DSA_MASK_CAUSAL, num_seqs=4, cu_seqlens=1 << 20,
+                      flags=F)                       # no host copy to size it from
+    with pytest.raises(dsa.DsaError) as e:
+        dsa.dsa_indexer_workspace_size(d)
+    assert e.value.status == dsa.DSA_ERR_INVALID_ARG
+    with pytest.raises(dsa.DsaError) as e:           # an unknown flag bit
+        dsa.dsa_indexer_workspace_size(good_desc(flags=4))
+    assert e.value.status == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_topk_only_forward_host_checks():
+    """scores = NULL needs the flag and a workspace that holds the rows;
+    both are checked before any device work."""
+    fake = 1 << 20
+    with pytest.raises(dsa.DsaError) as e:           # no flag
+        dsa.dsa_indexer_forward(good_desc(), fake, None, fake, fake, None, fake,
+                                None, fake, fake, 1 << 20)
+    assert e.value.status == dsa.DSA_ERR_INVALID_ARG
+    d = good_desc(flags=dsa.DSA_FLAG_SCORES_IN_WORKSPACE)
+    need = dsa.dsa_indexer_workspace_size(d)
+    with pytest.raises(dsa.DsaError) as e:           # workspace one float short
+        dsa.dsa_indexer_forward(d, fake, None, fake, fake, None, fake,
+                                None, fake, fake, need - 4)
+    assert e.value.status == dsa.DSA_ERR_WORKSPACE
+    with pytest.raises(dsa.DsaError) as e:           # noalloc has no room for rows
+        dsa.dsa_indexer_forward_noalloc(d, fake, None, fake, fake, None, fake, None, fake)
+    assert e.value.status in (dsa.DSA_ERR_INVALID_ARG, dsa.DSA_ERR_WORKSPACE)

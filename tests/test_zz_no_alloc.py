@@ -10,22 +10,22 @@ import pytest
 import torch
 
 import dsa_synth as syn
-from parity_util import TOL_BF16
+from parity_util import TOL_BF16, TOL_FP8
 
 pytestmark = pytest.mark.gpu
 
 
-def _compare(ref_scores, ref_topk, scores, topk):
+def _compare(ref_scores, ref_topk, scores, topk, tol=TOL_BF16):
     r, g = ref_scores.double().cpu().numpy(), scores.double().cpu().numpy()
     scale = np.abs(r[r > -1e38]).max()
-    assert np.abs(g - r).max() <= TOL_BF16 * scale
+    assert np.abs(g - r).max() <= tol * scale
     masked = r < -1e38
     assert np.array_equal(g[masked], r[masked])
     assert np.array_equal(np.sort(ref_topk.cpu().numpy(), axis=1),
                           np.sort(topk.cpu().numpy(), axis=1))
 
 
-@pytest.mark.parametrize("name", ["tiny_decode", "decode_batch"])
+@pytest.mark.parametrize("name", ["tiny_decode", "decode_batch", "long_decode_fp8"])
 def test_noalloc_matches_forward_twice(name):
     assert torch.cuda.is_available()
     import sparse_attention_lightning_tcgen05_b200 as dsa
@@ -42,7 +42,8 @@ def test_noalloc_matches_forward_twice(name):
                                         dp.k_cache, dp.k_scale, dp.positions,
                                         scores, topk, stream)
         torch.cuda.synchronize()
-        _compare(dp.scores, dp.topk, scores, topk)
+        _compare(dp.scores, dp.topk, scores, topk,
+                 TOL_FP8 if wl.dtype == syn.DTYPE_FP8 else TOL_BF16)
 
 
 def test_noalloc_causal_matches_forward():

@@ -51,6 +51,7 @@ DEFAULTS = {   # steps, warmup, graph length
     "decode_batch": (60000, 3000, 240),
     "decode_batch_paged": (60000, 3000, 240),
     "long_decode_fp8": (6000, 300, 60),
+    "long_decode_fp8_paged": (6000, 300, 60),
     "prefill_causal": (1500, 30, 30),
     "ragged_prefill": (20, 3, 1),
     "c4_prefill": (1500, 30, 30),
@@ -520,13 +521,122 @@ def workload_config(wl, extra=None):
     return c
 
 
+# ---------------------------------------------------------------- sparse MQA
+MQA_METRIC = "sparse-MQA (query token, kept key) pairs/s at 1 B200, % of roofline"
+MQA_DEFAULTS = {"mqa_decode": (20000, 1000, 200), "mqa_prefill": (200, 10, 10)}
+
+
+def mqa_algorithmic(wl, idx):
+    """(flops, bytes, kept entries) per step. FLOPs: 2*H*D for the logits and
+    2*H*D for the weighted sum, per kept entry. Bytes: q, the index rows, the
+    output, and every kv row some token of its batch selects, once."""
+    kept = (idx >= 0) & (idx < wl.K)
+    n_kept = int(kept.sum())
+    uniq = sum(int(np.unique(idx[b][kept[b]]).size) for b in range(wl.B))
+    T = wl.B * wl.S
+    nbytes = T * wl.H * wl.D * 2 * 2 + idx.size * 4 + uniq * wl.D * 2
+    return 4.0 * wl.H * wl.D * n_kept, nbytes, n_kept
+
+
+def run_mqa(args, wl):
+    import torch
+    import sparse_attention_lightning_tcgen05_b200 as m
+    from oracle.sparse_mqa import sparse_mqa
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    inputs = syn.generate_mqa(wl)
+    flops, nbytes, n_kept = mqa_algorithmic(wl, inputs["idx"])
+    T = wl.B * wl.S
+    desc = m.make_mqa_desc(wl.B, wl.S, wl.H, wl.K, wl.K_top, wl.sm_scale)
+    nsets = 1 if nbytes > 2 * L2_BYTES else min(8, int(np.ceil(2 * L2_BYTES / nbytes)) + 1)
+    ws_bytes = m.dsa_sparse_mqa_workspace_size(desc)
+    sets = []
+    for _ in range(nsets):
+        sets.append(dict(
+            q=torch.from_numpy(inputs["q"].view(np.int16)).to(device),
+            kv=torch.from_numpy(inputs["kv"].view(np.int16)).to(device),
+            sinks=torch.from_numpy(inputs["sinks"]).to(device),
+            idx=torch.from_numpy(inputs["idx"]).to(device),
+            out=torch.empty((wl.B, wl.S, wl.H, wl.D), dtype=torch.int16, device=device),
+            ws=torch.zeros(ws_bytes, dtype=torch.uint8, device=device)))
+    stream = torch.cuda.Stream(device=device)
+
+    def call(st):
+        return lambda: m.dsa_sparse_mqa_forward(desc, st["q"], st["kv"], st["sinks"], st["idx"],
+                                                st["out"], st["ws"], ws_bytes, stream.cuda_stream)
+    with torch.cuda.stream(stream):
+        for st in sets:
+            call(st)()
+    for st in sets:
+        assert m.dsa_indexer_get_error(st["ws"], stream.cuda_stream) == m.DSA_OK
+    glen = MQA_DEFAULTS[wl.name][2]
+    glen = max(nsets, glen // nsets * nsets)
+    steps, warmup = args.steps, args.warmup
+
+    def graphs(n):
+        main = capture([call(sets[i % nsets]) for i in range(min(glen, n))], stream)
+        rem = n % min(glen, n)
+        extra = [capture([call(sets[i % nsets]) for i in range(rem)], stream)] if rem else []
+        return [main] + extra, n // min(glen, n)
+    wg, wr = graphs(warmup)
+    w_ms = time_graphs(wg, wr, stream)
+    fg, fr = graphs(steps)
+    windows = int(min(50, max(1, np.ceil(500.0 / max(w_ms / warmup * steps, 1e-3)))))
+    uuid = str(torch.cuda.get_device_properties(device).uuid)
+    torch.cuda.synchronize(device)
+    with ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid) as clk:
+        ms_w = time_graphs(fg, fr, stream, windows)
+    ms_w = [ms_w] if windows == 1 else ms_w
+    ms = float(np.median(ms_w)) / steps
+    pk = peaks()
+    t_flops = flops / (pk["bf16"] * 1e12)
+    t_bytes = nbytes / (pk["hbm"] * 1e9)
+    bound = "tensor" if t_flops >= t_bytes else "hbm"
+    if bound == "tensor":
+        roof = {"bound": "tensor", "achieved": flops / (ms / 1e3) / 1e12, "peak": pk["bf16"],
+                "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": nbytes / (ms / 1e3) / 1e9, "peak": pk["hbm"],
+                "unit": "GB/s"}
+    roof.update(frac=roof["achieved"] / roof["peak"], traffic=None, kernel="sparse_mqa_kernel",
+                roofline_ms=max(t_flops, t_bytes) * 1e3,
+                peak_source=f"{pk['src']} (MEASURED_PEAKS.json)")
+    # the fp64 oracle on a bounded sample of tokens
+    cores = os.cpu_count() or 1
+    rng = np.random.default_rng(0)
+    toks = sorted(set(int(x) for x in rng.integers(0, T, min(T, 8))))
+    t0 = time.perf_counter()
+    for tk in toks:
+        b, s_ = divmod(tk, wl.S)
+        sparse_mqa(inputs["q"][b:b + 1, s_:s_ + 1], inputs["kv"][b:b + 1], inputs["sinks"],
+                   inputs["idx"][b:b + 1, s_:s_ + 1], wl.sm_scale)
+    dt = time.perf_counter() - t0
+    kept_t = sum(int(((inputs["idx"].reshape(T, -1)[tk] >= 0) &
+                      (inputs["idx"].reshape(T, -1)[tk] < wl.K)).sum()) for tk in toks)
+    return {"metric": MQA_METRIC, "value": n_kept / (ms / 1e3), "unit": "pairs/s", "n_gpus": 1,
+            "steps": steps, "warmup": warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "B": wl.B, "S": wl.S, "H": wl.H, "D": wl.D,
+                       "K": wl.K, "K_top": wl.K_top, "causal_index_rows": wl.causal},
+            "timing": {"l2": f"{nsets} rotating input copies" if nsets > 1
+                       else "inputs larger than L2", "windows": windows,
+                       "ms_per_step_windows": [x / steps for x in ms_w]},
+            "kept_pairs_per_step": n_kept, "tflops": flops / (ms / 1e3) / 1e12,
+            "roofline": roof, "clocks": clk.summary(),
+            "gpu_launches": (2 if ws_bytes > 256 else 1) * steps * windows,
+            "cpu_baseline": {"value": kept_t / dt, "unit": "pairs/s", "cores": 1,
+                             "kind": "oracle",
+                             "sample": f"{len(toks)} of {T} tokens (numpy fp64), {dt:.2f} s"}}
+
+
 # ---------------------------------------------------------------- main
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=None)
-    ap.add_argument("--workload", default="ragged_prefill", choices=sorted(syn.WORKLOADS))
+    ap.add_argument("--workload", default="ragged_prefill",
+                    choices=sorted(syn.WORKLOADS) + sorted(syn.MQA_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=None,
                     help="end-to-end steps (default 20; 5 for the ragged prefill)")
@@ -535,6 +645,17 @@ def main(argv=None):
                     help="packed causal workloads: other sequence lengths, comma "
                          "separated (a smaller batch of the same kind, for profiling)")
     args = ap.parse_args(argv)
+    if args.workload in syn.MQA_WORKLOADS:
+        wl = syn.MQA_WORKLOADS[args.workload]
+        d_steps, d_warm, _ = MQA_DEFAULTS[wl.name]
+        args.steps = d_steps if args.steps is None else args.steps
+        args.warmup = d_warm if args.warmup is None else args.warmup
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the oracle arm covers the "
+                              "indexer workloads only"}), flush=True)
+            return 0
+        print(json.dumps(run_mqa(args, wl)), flush=True)
+        return 0
     wl = syn.WORKLOADS[args.workload]
     if args.seqlens:
         if wl.mode != syn.MODE_CAUSAL:

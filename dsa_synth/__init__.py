@@ -126,6 +126,12 @@ WORKLOADS = {
     "decode_batch_paged": Workload("decode_batch_paged", MODE_POSITIONS, T=16, H=64,
                                    D=128, index_topk=2048, S=32768, pos_lo=2048,
                                    pos_hi=32768, w_scale=1.0 / 8.0, page_size=64),
+    # the long-context fp8 decode over a paged cache: 64-slot pages of e4m3
+    # keys and of their e8m0 scale rows, scattered by a random block table
+    "long_decode_fp8_paged": Workload("long_decode_fp8_paged", MODE_POSITIONS, T=64,
+                                      H=64, D=128, index_topk=1024, dtype=DTYPE_FP8,
+                                      S=131072, pos_lo=1024, pos_hi=131072,
+                                      w_scale=1.0 / 8.0, page_size=64),
     # compressed (C4) indexer, the next step beyond the five: an 8192-token
     # prefill chunk against its 2048 keys pooled 4:1, DSV4's index_topk 1024
     "c4_prefill": Workload("c4_prefill", MODE_COMPRESSED, T=8192, H=64, D=128,
@@ -271,3 +277,66 @@ def generate(wl: Workload, value_kind: str = "gauss",
     elif wl.mode == MODE_CAUSAL:
         out["cu_seqlens"] = wl.cu_seqlens()
     return out
+
+
+# ---- the indexer's consumer: sparse MQA over top-k key indices ----------------
+
+@dataclasses.dataclass(frozen=True)
+class MqaWorkload:
+    """One synthetic sparse-MQA problem: q [B,S,H,D], one kv head [B,K,D],
+    sinks [H], index rows [B,S,K_top] (NeMo AutoModel optimized_kernels,
+    sparse_attention_torch)."""
+    name: str
+    B: int
+    S: int
+    H: int
+    K: int
+    K_top: int
+    D: int = 128
+    causal: bool = False        # token s of a batch picks among keys [0, s]
+    seed: int = 0
+
+    @property
+    def sm_scale(self) -> float:
+        return float(self.D) ** -0.5
+
+
+MQA_WORKLOADS = {
+    # the decode batch's consumer: one token per sequence, its 2048 selected
+    # slots of a 32768-slot cache
+    "mqa_decode": MqaWorkload("mqa_decode", B=16, S=1, H=64, K=32768, K_top=2048),
+    # the causal prefill's consumer: 8192 tokens, each its 2048 selected keys
+    # among the ones at or before it (-1 padded below 2048 visible keys)
+    "mqa_prefill": MqaWorkload("mqa_prefill", B=1, S=8192, H=64, K=8192, K_top=2048,
+                               causal=True),
+}
+
+
+def generate_mqa(wl: MqaWorkload, seed: Optional[int] = None) -> dict:
+    """Draw a sparse-MQA problem (host arrays, storage formats).
+
+    ``numpy.random.default_rng(seed)``, draws in the order q, kv, sinks,
+    index rows. q, kv ~ N(0,1) as bf16 bits; sinks ~ N(0,1) float32. Each
+    token's index row holds K_top distinct key rows drawn uniformly from the
+    keys it may see (all K, or [0, s] for a causal batch), in random order,
+    -1 padded when it sees fewer than K_top keys -- the form of the indexer's
+    top-k sets."""
+    rng = np.random.default_rng(wl.seed if seed is None else seed)
+    B, S, H, D, K = wl.B, wl.S, wl.H, wl.D, wl.K
+    q = f32_to_bf16_bits(gaussian_f32(rng, B * S * H * D).reshape(B, S, H, D))
+    kv = f32_to_bf16_bits(gaussian_f32(rng, B * K * D).reshape(B, K, D))
+    sinks = gaussian_f32(rng, H)
+    idx = np.full((B, S, wl.K_top), -1, np.int32)
+    for b in range(B):
+        for s in range(S):
+            n = min(K, s + 1) if wl.causal else K
+            m = min(n, wl.K_top)
+            if n <= 4 * wl.K_top:
+                pick = rng.permutation(n)[:m]
+            else:                   # sample without a full permutation of n
+                pick = np.unique(rng.integers(0, n, size=2 * m))
+                while pick.size < m:
+                    pick = np.unique(np.concatenate([pick, rng.integers(0, n, size=m)]))
+                pick = rng.permutation(pick)[:m]
+            idx[b, s, :m] = pick
+    return dict(q=q, kv=kv, sinks=sinks, idx=idx)

@@ -135,11 +135,13 @@ typedef struct {
   int32_t pages_per_seq;   /* paged: block-table entries per token, >= 1, with
                               S <= pages_per_seq * page_size                    */
   int32_t num_pages;       /* paged: pages in the pool k points to, >= 1        */
-  const int32_t *block_table; /* NULL: not paged. Paged (POSITIONS, bf16 only,
+  const int32_t *block_table; /* NULL: not paged. Paged (POSITIONS,
                               k_seq_stride 0): device [T, pages_per_seq] int32;
                               token t's slot s is row s % page_size of page
                               block_table[t*pages_per_seq + s/page_size] of the
-                              pool k [num_pages, page_size, D]. Entries of pages
+                              pool k [num_pages, page_size, D] (FP8: and of the
+                              scale pool k_scale [num_pages, page_size, D/32],
+                              the same page ids). Entries of pages
                               that hold a valid slot must lie in
                               [0, num_pages); other entries are never used for
                               a score (a page id outside the pool reads as 0)  */
@@ -180,7 +182,8 @@ typedef struct {
  *           CAUSAL:    [T, D], sequence i at rows cu[i] .. cu[i+1]-1
  *           bf16, or e4m3 bytes                                 (16-byte aligned)
  *  k_scale  same slots as k, [.., D/32] e8m0 bytes (FP8 only; NULL for BF16);
- *           POSITIONS cache t at byte t*(k_seq_stride/32)
+ *           POSITIONS cache t at byte t*(k_seq_stride/32); paged: the scale
+ *           page pool [num_pages, page_size, D/32]          (16-byte aligned)
  *  positions [T] int32 (POSITIONS only; ignored for CAUSAL; must be NULL
  *           for COMPRESSED). A negative position leaves the whole row masked.
  *  scores   POSITIONS, COMPRESSED: [T, S] fp32 (a COMPRESSED row that sees

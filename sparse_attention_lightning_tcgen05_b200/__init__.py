@@ -32,10 +32,11 @@ DSA_MASK_BOUND = float.fromhex("-0x1.FEp127")
 DSA_FLAG_SCORES_IN_WORKSPACE = 1
 DSA_FLAG_SELFTEST_STALL = 2
 
-# Every symbol include/dsa_indexer.h declares.
+# Every symbol include/dsa_indexer.h and include/dsa_sparse_mqa.h declare.
 EXPORTS = ("dsa_indexer_workspace_size", "dsa_indexer_score", "dsa_indexer_topk",
            "dsa_indexer_forward", "dsa_indexer_forward_noalloc",
-           "dsa_indexer_get_error", "dsa_status_string")
+           "dsa_indexer_get_error", "dsa_sparse_mqa_workspace_size",
+           "dsa_sparse_mqa_forward", "dsa_status_string")
 
 
 class dsa_indexer_desc_t(ctypes.Structure):
@@ -49,6 +50,12 @@ class dsa_indexer_desc_t(ctypes.Structure):
                 ("num_pages", ctypes.c_int32), ("block_table", ctypes.c_void_p),
                 ("flags", ctypes.c_uint32), ("wait_limit_ns", ctypes.c_uint64),
                 ("cu_seqlens_host", ctypes.c_void_p)]
+
+
+class dsa_sparse_mqa_desc_t(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("S", ctypes.c_int32), ("H", ctypes.c_int32),
+                ("D", ctypes.c_int32), ("K", ctypes.c_int64), ("K_top", ctypes.c_int32),
+                ("sm_scale", ctypes.c_float), ("wait_limit_ns", ctypes.c_uint64)]
 
 
 class DsaError(RuntimeError):
@@ -73,6 +80,9 @@ _lib.dsa_indexer_topk.argtypes = [_P, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.dsa_indexer_forward.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.dsa_indexer_forward_noalloc.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 _lib.dsa_indexer_get_error.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_int)]
+_M = ctypes.POINTER(dsa_sparse_mqa_desc_t)
+_lib.dsa_sparse_mqa_workspace_size.argtypes = [_M, ctypes.POINTER(_sz)]
+_lib.dsa_sparse_mqa_forward.argtypes = [_M, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 _lib.dsa_status_string.argtypes = [ctypes.c_int]
 _lib.dsa_status_string.restype = ctypes.c_char_p
 for _f in EXPORTS[:-1]:
@@ -178,3 +188,22 @@ def current_stream_handle():
     """The cudaStream_t of torch's current CUDA stream."""
     import torch
     return torch.cuda.current_stream().cuda_stream
+
+
+def make_mqa_desc(B, S, H, K, K_top, sm_scale, *, D=128, wait_limit_ns=0):
+    return dsa_sparse_mqa_desc_t(B=B, S=S, H=H, D=D, K=K, K_top=K_top,
+                                 sm_scale=sm_scale, wait_limit_ns=wait_limit_ns)
+
+
+def dsa_sparse_mqa_workspace_size(desc) -> int:
+    n = _sz(0)
+    _check(_lib.dsa_sparse_mqa_workspace_size(ctypes.byref(desc), ctypes.byref(n)),
+           "dsa_sparse_mqa_workspace_size")
+    return n.value
+
+
+def dsa_sparse_mqa_forward(desc, q, kv, sinks, topk, out, workspace, workspace_bytes,
+                           stream=None) -> int:
+    return _check(_lib.dsa_sparse_mqa_forward(
+        ctypes.byref(desc), _ptr(q), _ptr(kv), _ptr(sinks), _ptr(topk), _ptr(out),
+        _ptr(workspace), workspace_bytes, stream), "dsa_sparse_mqa_forward")

@@ -44,12 +44,6 @@ static_assert(sizeof(WsHeader) == kWorkspaceHeader, "header size");
 
 // ---- per-device state -----------------------------------------------------------
 
-struct DeviceInfo {
-  bool probed = false;
-  bool ok = false;
-  int num_sms = 0;
-  uint32_t attr_done = 0;   // bit per kernel whose smem attribute is set
-};
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -85,8 +79,7 @@ dsa_status_t device_info(DeviceInfo **out) {
 }
 
 // Raise the dynamic shared-memory limit of kernel `bit` once per device.
-template <typename K>
-dsa_status_t ensure_smem_attr(DeviceInfo *d, uint32_t bit, K kernel, int bytes) {
+dsa_status_t ensure_smem_attr_raw(DeviceInfo *d, uint32_t bit, const void *kernel, int bytes) {
   std::lock_guard<std::mutex> lk(g_mu);
   if (d->attr_done >> bit & 1u) return DSA_OK;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
@@ -97,8 +90,6 @@ dsa_status_t ensure_smem_attr(DeviceInfo *d, uint32_t bit, K kernel, int bytes) 
 }
 
 // ---- argument checks -----------------------------------------------------------------
-
-bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 dsa_status_t check_desc(const dsa_indexer_desc_t *d) {
   if (!d) return DSA_ERR_INVALID_ARG;
@@ -121,7 +112,6 @@ dsa_status_t check_desc(const dsa_indexer_desc_t *d) {
     if (d->S < 1 || d->S > static_cast<int64_t>(d->pages_per_seq) * d->page_size)
       return DSA_ERR_INVALID_ARG;
     if (!aligned(d->block_table, 4)) return DSA_ERR_INVALID_ARG;
-    if (d->dtype != DSA_KV_BF16) return DSA_ERR_UNSUPPORTED;
   }
   if (d->mask == DSA_MASK_POSITIONS) {
     if (d->S < 1) return DSA_ERR_INVALID_ARG;
@@ -192,8 +182,7 @@ int64_t workspace_scores(void *ws, size_t ws_bytes, float **scores) {
 
 dsa_status_t make_map(CUtensorMap *m, CUtensorMapDataType dt, cuuint32_t rank, const void *base,
                       const cuuint64_t *dims, const cuuint64_t *strides_bytes,
-                      const cuuint32_t *box,
-                      CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
+                      const cuuint32_t *box, CUtensorMapSwizzle swz) {
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(m, dt, rank, const_cast<void *>(base), dims, strides_bytes, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
@@ -216,32 +205,7 @@ struct ScoreLaunch {
   int threads() const { return (2 + epi + (fp8 ? 1 : 0) + (issuers - 1)) * 32; }
 };
 
-// Launch with programmatic stream serialisation: the kernel may start while
-// the previous kernel on the stream is finishing; each kernel calls
-// griddepcontrol.wait before it touches memory that earlier work wrote.
-// `cluster` > 0 launches thread-block clusters of that many CTAs along x.
-template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int threads, size_t smem,
-                       cudaStream_t stream, int cluster, Args &&...args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(static_cast<unsigned>(threads));
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cluster > 0) {
-    attr[1].id = cudaLaunchAttributeClusterDimension;
-    attr[1].val.clusterDim.x = static_cast<unsigned>(cluster);
-    attr[1].val.clusterDim.y = 1;
-    attr[1].val.clusterDim.z = 1;
-    cfg.numAttrs = 2;
-  }
-  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
-}
+
 
 int round16(int x) { return (x + 15) / 16 * 16; }
 
@@ -370,8 +334,20 @@ dsa_status_t launch_score(const dsa_indexer_desc_t *d, const void *q, const uint
     const cuuint64_t strides[2] = {128 * elt, ps * 128 * elt};
     const cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elt),
                                static_cast<cuuint32_t>(std::min<cuuint64_t>(ps, dsa::kBlockM)), 1};
-    st = make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, k, dims, strides, box);
+    st = make_map(&tk, L.fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                  k, dims, strides, box);
     if (st != DSA_OK) return st;
+    if (L.fp8) {
+      // the scale pool [num_pages, page_size] of 32-bit words (4 e8m0 bytes
+      // a slot), one box per page box of the data
+      const cuuint64_t sdims[2] = {ps, static_cast<cuuint64_t>(d->num_pages)};
+      const cuuint64_t sstrides[1] = {ps * 4};
+      const cuuint32_t sbox[2] = {static_cast<cuuint32_t>(std::min<cuuint64_t>(ps, dsa::kBlockM)),
+                                  1};
+      st = make_map(&tksf, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, k_scale, sdims, sstrides, sbox,
+                    CU_TENSOR_MAP_SWIZZLE_NONE);
+      if (st != DSA_OK) return st;
+    }
   } else {
     const cuuint64_t dims[3] = {128, rows, caches};
     const cuuint64_t strides[2] = {128 * elt, stride_elems * elt};
@@ -389,7 +365,7 @@ dsa_status_t launch_score(const dsa_indexer_desc_t *d, const void *q, const uint
                   q, dims, strides, box);
     if (st != DSA_OK) return st;
   }
-  if (L.fp8) {
+  if (L.fp8 && !paged) {
     // scale bytes of one slot (4 blocks of 32 along D) read as one 32-bit word
     // (one cache: the second dimension is never stepped; its stride only
     // has to be a legal multiple of 16 bytes)
@@ -399,6 +375,8 @@ dsa_status_t launch_score(const dsa_indexer_desc_t *d, const void *q, const uint
     st = make_map(&tksf, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, k_scale, dims, strides, box,
                   CU_TENSOR_MAP_SWIZZLE_NONE);
     if (st != DSA_OK) return st;
+  }
+  if (L.fp8) {
     const cuuint64_t qdims[2] = {qrows, 1};
     const cuuint64_t qstrides[1] = {(qrows * 4 + 15) / 16 * 16};   // never stepped
     const cuuint32_t qbox[2] = {static_cast<cuuint32_t>(L.n_cols + dsa::kSfPad), 1};

@@ -89,7 +89,11 @@ __host__ __device__ constexpr uint32_t round128(uint32_t x) { return (x + 127u) 
 // bytes one scale-window copy delivers (the mbarrier's expected transaction
 // count) and the shared-memory room it takes
 constexpr uint32_t kSfBoxBytesK = (kBlockM + kSfPad) * 4;
-constexpr uint32_t kSfRawBytesK = round128(kSfBoxBytesK);
+// A paged tile's scale words come one box per page; a TMA destination must be
+// 128-byte aligned, so 16-slot pages (64 bytes of words a box) each get a
+// 128-byte slot: 8 slots, 1024 bytes, which also holds the unpaged window.
+constexpr uint32_t kSfRawBytesK = 1024;
+static_assert(kSfRawBytesK >= round128(kSfBoxBytesK), "scale window room");
 __host__ __device__ constexpr uint32_t sf_box_bytes_q(int n_cols) {
   return static_cast<uint32_t>((n_cols + kSfPad) * 4);
 }
@@ -673,6 +677,19 @@ struct Ring {
 // fp8: reorder 128 rows of 4 scale bytes (row-major, as loaded) into the
 // scale-factor atom tcgen05.cp copies: row m = m0 + 32*m1 at byte
 // 16*m0 + 4*m1 (+ K block). Rows >= nrows read as 0. Full warp.
+// The same from the scale words of a paged tile with 16-slot pages: row m at
+// word 32 * (m / 16) + m % 16 (one 128-byte slot per page box). Full warp.
+__device__ __forceinline__ void sf_reorder_atom_pages16(const uint32_t *slots, uint32_t *atom) {
+  const int l = threadIdx.x & 31;
+  auto word = [&](int m) { return slots[((m >> 4) << 5) + (m & 15)]; };
+  uint4 v;
+  v.x = word(l);
+  v.y = word(l + 32);
+  v.z = word(l + 64);
+  v.w = word(l + 96);
+  reinterpret_cast<uint4 *>(atom)[l] = v;
+}
+
 __device__ __forceinline__ void sf_reorder_atom(const uint32_t *rows, int nrows,
                                                 uint32_t *atom) {
   const int l = threadIdx.x & 31;
@@ -812,7 +829,10 @@ __global__ void __launch_bounds__((2 + kEPI + (kFP8 ? 1 : 0) + (kISS - 1)) * 32,
       uint32_t k_issued = 0, q_issued = 0, k_last_phase = 0, q_last_phase = 0;
       ItemCursor c;
       cursor_start(P, tqt, R, c);
-      const uint32_t tile_tx = L.k_stage_bytes + (kFP8 ? kSfBoxBytesK : 0);
+      // fp8: a paged tile's scale words come page by page, each box at its
+      // row offset (no window padding: page boxes start on 4-word rows)
+      const uint32_t tile_tx =
+          L.k_stage_bytes + (kFP8 ? (p.block_table ? kBlockM * 4 : kSfBoxBytesK) : 0);
       bool need_q = true;
       while (c.left > 0) {
         const int g = cursor_tiles<kG>(c);
@@ -842,11 +862,14 @@ __global__ void __launch_bounds__((2 + kEPI + (kFP8 ? 1 : 0) + (kISS - 1)) * 32,
         for (int i = 0; i < g; ++i) {
           uint8_t *dst = sk + (st.idx * kG + i) * L.k_stage_bytes;
           const int y = c.q.y0 + (c.j + i) * kBlockM;
-          if (!kFP8 && p.block_table) {
+          if (p.block_table) {
             // paged cache: the tile's slots y .. y+127 from one page, or from
             // 128/page_size pages (one box each, at its row offset in the
             // tile; 128-byte swizzle atoms are 8 rows, boxes >= 16 rows).
             // Past the block table, an id past the pool: TMA fills zeros.
+            // fp8: each box's scale words land at the same row offset of the
+            // tile's scale window (a box starts on a page row that is a
+            // multiple of 16, so its words are 16-byte aligned).
             const int box = p.page_shift >= 7 ? kBlockM : (1 << p.page_shift);
             for (int b = 0; b < kBlockM; b += box) {
               const int lp = (y + b) >> p.page_shift;
@@ -856,7 +879,16 @@ __global__ void __launch_bounds__((2 + kEPI + (kFP8 ? 1 : 0) + (kISS - 1)) * 32,
                       ? __ldg(p.block_table + static_cast<int64_t>(c.q.z) * p.pages_per_seq + lp)
                       : p.num_pages;
               tma_load_3d(dst + b * 128, &tmap_k, full_k + st.idx, 0, row, page);
-              tma_load_3d(dst + kBlockM * 128 + b * 128, &tmap_k, full_k + st.idx, 64, row, page);
+              if constexpr (kFP8) {
+                // boxes of >= 32 rows: at their row offset (a multiple of 128
+                // bytes); 16-row boxes: one 128-byte slot each
+                const int sf_off = box >= 32 ? 4 * b : 8 * b;
+                tma_load_2d(sksf + (st.idx * kG + i) * L.k_sf_bytes + sf_off, &tmap_ksf,
+                            full_k + st.idx, row, page);
+              } else {
+                tma_load_3d(dst + kBlockM * 128 + b * 128, &tmap_k, full_k + st.idx, 64, row,
+                            page);
+              }
             }
             continue;
           }
@@ -1029,8 +1061,12 @@ __global__ void __launch_bounds__((2 + kEPI + (kFP8 ? 1 : 0) + (kISS - 1)) * 32,
         for (int i = 0; i < g; ++i) {
           uint8_t *sf = sksf + (st.idx * kG + i) * L.k_sf_bytes;
           const int r = (c.q.y0 + (c.j + i) * kBlockM) & (kSfPad - 1);
-          sf_reorder_atom(reinterpret_cast<const uint32_t *>(sf) + r, 128,
-                          reinterpret_cast<uint32_t *>(sf + kSfRawBytesK));
+          if (p.block_table && p.page_shift < 5)
+            sf_reorder_atom_pages16(reinterpret_cast<const uint32_t *>(sf),
+                                    reinterpret_cast<uint32_t *>(sf + kSfRawBytesK));
+          else
+            sf_reorder_atom(reinterpret_cast<const uint32_t *>(sf) + r, 128,
+                            reinterpret_cast<uint32_t *>(sf + kSfRawBytesK));
         }
         fence_proxy_async_smem();
         __syncwarp();

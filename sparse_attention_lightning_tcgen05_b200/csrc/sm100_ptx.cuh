@@ -173,7 +173,7 @@ constexpr unsigned int kStatusTimeout = 5;   // == DSA_ERR_TIMEOUT
 // outlives ctl.limit_ns or another role of the CTA has aborted. Never spins
 // without a bound: the time check runs every 64 polls and the poll count is
 // capped as a second bound.
-__device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
+static __device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
                                        const WaitCtl &ctl, uint32_t site) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
@@ -192,7 +192,7 @@ __device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
 
 // Same as mbar_wait but ignores the abort flag: used on the way out, to let
 // copies or MMAs that are still in flight land before the CTA exits.
-__device__ __noinline__ void mbar_drain(uint64_t *bar, uint32_t parity,
+static __device__ __noinline__ void mbar_drain(uint64_t *bar, uint32_t parity,
                                         uint64_t limit_ns) {
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 0; i < (1u << 30); ++i) {
@@ -502,6 +502,74 @@ __device__ __forceinline__ void tmem_ld64_wait(uint32_t taddr, uint32_t (&r)[64]
         "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
       : "r"(taddr)
       : "memory");
+}
+
+}  // namespace dsa
+
+namespace dsa {
+
+// ---- helpers of the sparse-MQA kernel --------------------------------------------
+
+// 16-byte asynchronous copy global -> shared that writes zeros instead when
+// src_bytes == 0 (the source is then not read).
+__device__ __forceinline__ void cp_async16_zfill(void *smem_dst, const void *gmem_src,
+                                                 uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)),
+               "l"(gmem_src), "r"(src_bytes)
+               : "memory");
+}
+
+// 2^x (hardware approximation, flush-to-zero; 2^-inf = 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// MN-major operand with 128-byte swizzle: rows of 128 bytes run
+// along MN (64 16-bit elements), 8 consecutive K rows form a 1024-byte atom.
+// lbo_bytes: distance between atoms along MN (the next 64 MN elements),
+// sbo_bytes: distance between atoms along K (the next 8 K rows).
+__device__ __forceinline__ uint64_t sdesc_mnmajor_sw128(uint32_t saddr, uint32_t lbo_bytes,
+                                                        uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);              // start address
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;    // LBO
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;    // SBO
+  d |= static_cast<uint64_t>(1u) << 46;                            // sm100 version
+  d |= static_cast<uint64_t>(2u) << 61;                            // 128B swizzle
+  return d;
+}
+
+// Instruction descriptor of kind::f16, bf16 A (K-major) and bf16 B
+// (MN-major), fp32 D.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_bmn(uint32_t M, uint32_t N) {
+  return idesc_bf16_f32(M, N) | (1u << 16);
+}
+
+// 32 TMEM lanes x 32 consecutive 32-bit columns <- 32 registers per thread.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+      ::"r"(taddr),
+        "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]),
+        "f"(v[7]), "f"(v[8]), "f"(v[9]), "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]),
+        "f"(v[14]), "f"(v[15]), "f"(v[16]), "f"(v[17]), "f"(v[18]), "f"(v[19]), "f"(v[20]),
+        "f"(v[21]), "f"(v[22]), "f"(v[23]), "f"(v[24]), "f"(v[25]), "f"(v[26]), "f"(v[27]),
+        "f"(v[28]), "f"(v[29]), "f"(v[30]), "f"(v[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Arrive on `bar` once every cp.async this thread issued so far has landed
+// (the arrival counts toward the barrier's expected count).
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t *bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
 }
 
 }  // namespace dsa

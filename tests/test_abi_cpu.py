@@ -10,12 +10,17 @@ import sparse_attention_lightning_tcgen05_b200 as dsa
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "dsa_indexer.h")
+HEADERS = [os.path.join(ROOT, "include", f) for f in sorted(os.listdir(os.path.join(ROOT, "include")))
+           if f.endswith(".h")]
 
 
 def declared_functions():
-    src = open(HEADER).read()
-    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(dsa_\w+)\s*\(", src)))
+    names = set()
+    for h in HEADERS:
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names.update(re.findall(r"\b(dsa_\w+)\s*\(", src))
+    return sorted(names)
 
 
 def test_exports_every_declared_symbol():
@@ -110,6 +115,7 @@ def test_paged_descriptor_layout():
     assert f.block_table.offset % 8 == 0 and f.block_table.offset == f.num_pages.offset + 4
     assert dsa.dsa_indexer_workspace_size(paged_desc()) >= 256
     assert dsa.dsa_indexer_workspace_size(paged_desc(page_size=16, pages_per_seq=63)) >= 256
+    assert dsa.dsa_indexer_workspace_size(paged_desc(dtype=dsa.DSA_KV_FP8_E4M3_E8M0_B32)) >= 256
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -121,7 +127,6 @@ def test_paged_descriptor_layout():
     (dict(k_seq_stride=1000 * 128), dsa.DSA_ERR_INVALID_ARG),   # a pool, not per-token caches
     (dict(mask=dsa.DSA_MASK_CAUSAL, num_seqs=1, cu_seqlens=1 << 20), dsa.DSA_ERR_INVALID_ARG),
     (dict(block_table=(1 << 20) + 2), dsa.DSA_ERR_INVALID_ARG),   # misaligned table
-    (dict(dtype=dsa.DSA_KV_FP8_E4M3_E8M0_B32), dsa.DSA_ERR_UNSUPPORTED),
 ])
 def test_bad_paged_descriptors(kw, code):
     with pytest.raises(dsa.DsaError) as e:
@@ -326,3 +331,32 @@ def test_topk_only_forward_host_checks():
     with pytest.raises(dsa.DsaError) as e:           # noalloc has no room for rows
         dsa.dsa_indexer_forward_noalloc(d, fake, None, fake, fake, None, fake, None, fake)
     assert e.value.status in (dsa.DSA_ERR_INVALID_ARG, dsa.DSA_ERR_WORKSPACE)
+
+
+
+def test_sparse_mqa_host_checks():
+    """The sparse-MQA entry points check the descriptor and pointers on the
+    host, and size the workspace from the descriptor alone: the header, plus
+    the partial results when too few tokens fill the GPU and index rows are
+    split into ranges."""
+    d = dsa.make_mqa_desc(16, 1, 64, 32768, 2048, 128 ** -0.5)
+    n = dsa.dsa_sparse_mqa_workspace_size(d)
+    # 16 tokens: each row split into 8 ranges of 256 entries
+    assert n == 256 + 16 * 8 * 64 * 130 * 4
+    assert dsa.dsa_sparse_mqa_workspace_size(dsa.make_mqa_desc(1, 8192, 64, 8192, 2048, 0.1)) == 256
+    for kw, code in ((dict(H=0), dsa.DSA_ERR_INVALID_ARG), (dict(H=129), dsa.DSA_ERR_UNSUPPORTED),
+                     (dict(D=64), dsa.DSA_ERR_UNSUPPORTED), (dict(K_top=0), dsa.DSA_ERR_INVALID_ARG),
+                     (dict(sm_scale=float("nan")), dsa.DSA_ERR_INVALID_ARG)):
+        args = dict(B=2, S=3, H=8, K=100, K_top=64, sm_scale=0.1)
+        args.update(kw)
+        with pytest.raises(dsa.DsaError) as e:
+            dsa.dsa_sparse_mqa_workspace_size(dsa.make_mqa_desc(**args))
+        assert e.value.status == code
+    fake = 1 << 20
+    d = dsa.make_mqa_desc(2, 3, 8, 100, 64, 0.1)
+    with pytest.raises(dsa.DsaError) as e:               # misaligned q
+        dsa.dsa_sparse_mqa_forward(d, fake + 2, fake, fake, fake, fake, fake, 256)
+    assert e.value.status == dsa.DSA_ERR_INVALID_ARG
+    with pytest.raises(dsa.DsaError) as e:               # workspace too small
+        dsa.dsa_sparse_mqa_forward(d, fake, fake, fake, fake, fake, fake, 128)
+    assert e.value.status == dsa.DSA_ERR_WORKSPACE

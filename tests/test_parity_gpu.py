@@ -279,9 +279,9 @@ def test_decode_topk_row_lengths(dsa, S):
 
 # ---- paged key caches (block tables) ------------------------------------------
 
-def paged_wl(T, H, S, k, page, seed=0):
+def paged_wl(T, H, S, k, page, seed=0, dtype=syn.DTYPE_BF16):
     return syn.Workload("pg", syn.MODE_POSITIONS, T=T, H=H, D=128, index_topk=k, S=S,
-                        pos_lo=0, pos_hi=S, page_size=page,
+                        pos_lo=0, pos_hi=S, page_size=page, dtype=dtype,
                         w_scale=1.0 / np.sqrt(H), seed=seed)
 
 
@@ -332,3 +332,43 @@ def test_paged_single_large_page(dsa):
     """One page holds the whole cache (pages of 4096 slots, S = 3000)."""
     wl = paged_wl(T=3, H=64, S=3000, k=100, page=4096, seed=81)
     run_and_check(dsa, wl, syn.generate(wl))
+
+
+# ---- paged fp8 caches: e4m3 pages and their e8m0 scale pages ------------------
+
+@pytest.mark.parametrize("page", [16, 32, 64, 128, 256, 1024])
+def test_paged_fp8_decode(dsa, page):
+    """Pages smaller than a key tile (several data and scale boxes a tile),
+    equal to it and larger; S not a multiple of the page."""
+    wl = paged_wl(T=5, H=64, S=1000, k=64, page=page, seed=90 + page, dtype=syn.DTYPE_FP8)
+    run_and_check(dsa, wl, syn.generate(wl), tol=TOL_FP8)
+
+
+def test_paged_fp8_integer_bit_exact(dsa):
+    wl = paged_wl(T=4, H=64, S=700, k=40, page=32, seed=91, dtype=syn.DTYPE_FP8)
+    run_and_check(dsa, wl, syn.generate(wl, value_kind="int"), tol=TOL_FP8, exact=True)
+
+
+def test_paged_fp8_generic_heads(dsa):
+    wl = paged_wl(T=6, H=16, S=900, k=50, page=64, seed=92, dtype=syn.DTYPE_FP8)
+    run_and_check(dsa, wl, syn.generate(wl), tol=TOL_FP8)
+
+
+def test_paged_fp8_unused_table_entries(dsa):
+    """Table entries past a token's position (-1, far past the pool) are
+    never used for a score, in the data pool or the scale pool."""
+    wl = paged_wl(T=6, H=64, S=1200, k=64, page=64, seed=93, dtype=syn.DTYPE_FP8)
+    inputs = syn.generate(wl)
+    inputs["positions"] = np.array([0, 63, 64, 500, 1199, 129], np.int32)
+    bt = inputs["block_table"].copy()
+    for t, pos in enumerate(inputs["positions"]):
+        bt[t, pos // 64 + 1:] = np.where(np.arange(bt.shape[1] - pos // 64 - 1) % 2, -1, 1 << 30)
+    inputs["block_table"] = bt
+    run_and_check(dsa, wl, inputs, tol=TOL_FP8)
+
+
+def test_long_decode_fp8_paged_full_size_sampled(dsa):
+    wl = syn.WORKLOADS["long_decode_fp8_paged"]
+    rng = np.random.default_rng(16)
+    rows = sorted(set([0, 1, 63] + list(rng.integers(0, wl.T, 9))))
+    run_and_check(dsa, wl, syn.generate(wl), rows=rows, tol=TOL_FP8)

@@ -629,6 +629,115 @@ def run_mqa(args, wl):
                              "sample": f"{len(toks)} of {T} tokens (numpy fp64), {dt:.2f} s"}}
 
 
+# ---------------------------------------------------------------- the front end
+PREP_METRIC = "indexer front end (q, k, w projections) tokens/s at 1 B200, % of roofline"
+PREP_DEFAULTS = {"prepare_decode": (20000, 1000, 200), "prepare_prefill": (200, 10, 10)}
+
+
+def prep_algorithmic(wl):
+    """(flops, bytes) per step: the three projections' multiply-adds; the
+    weights, the activations and the outputs (q, k rows, w) moved once."""
+    T, H, D = wl.T, wl.H, wl.D
+    flops = 2.0 * T * (H * D * wl.q_lora_rank + (D + H) * wl.hidden)
+    weights = 2 * (H * D * wl.q_lora_rank + (D + H) * wl.hidden)
+    acts = 2 * T * (wl.hidden + wl.q_lora_rank)
+    outs = T * (H * D * 2 + H * 4 + D * 2)
+    return flops, weights + acts + outs
+
+
+def run_prepare(args, wl):
+    import torch
+    import sparse_attention_lightning_tcgen05_b200 as m
+    from oracle.front_end import front_end
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    inputs = syn.generate_prepare(wl)
+    flops, nbytes = prep_algorithmic(wl)
+    desc = m.make_prepare_desc(wl.T, wl.H, wl.hidden, wl.q_lora_rank, wl.rope_dim,
+                               w_scale=wl.w_scale)
+    ws_bytes = m.dsa_indexer_prepare_workspace_size(desc)
+    nsets = 1 if nbytes > 2 * L2_BYTES else min(8, int(np.ceil(2 * L2_BYTES / nbytes)) + 1)
+
+    def dev(a):
+        a = np.ascontiguousarray(a)
+        return torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a).to(device)
+    sets = []
+    for _ in range(nsets):
+        st = {k: dev(inputs[k]) for k in ("x", "qr", "wq_b", "wk", "wp", "gain", "bias",
+                                          "cos", "sin")}
+        st.update(q=torch.empty((wl.T, wl.H, wl.D), dtype=torch.int16, device=device),
+                  w=torch.empty((wl.T, wl.H), dtype=torch.float32, device=device),
+                  k=torch.empty((wl.T, wl.D), dtype=torch.int16, device=device),
+                  ws=torch.zeros(ws_bytes, dtype=torch.uint8, device=device))
+        sets.append(st)
+    stream = torch.cuda.Stream(device=device)
+
+    def call(st):
+        return lambda: m.dsa_indexer_prepare(desc, st["x"], st["qr"], st["wq_b"], st["wk"],
+                                             st["wp"], st["gain"], st["bias"], st["cos"],
+                                             st["sin"], None, st["q"], st["w"], st["k"],
+                                             st["ws"], ws_bytes, stream.cuda_stream)
+    with torch.cuda.stream(stream):
+        for st in sets:
+            call(st)()
+    for st in sets:
+        assert m.dsa_indexer_get_error(st["ws"], stream.cuda_stream) == m.DSA_OK
+    glen = PREP_DEFAULTS[wl.name][2]
+    glen = max(nsets, glen // nsets * nsets)
+    steps, warmup = args.steps, args.warmup
+
+    def graphs(n):
+        g = min(glen, n)
+        main = capture([call(sets[i % nsets]) for i in range(g)], stream)
+        rem = n % g
+        extra = [capture([call(sets[i % nsets]) for i in range(rem)], stream)] if rem else []
+        return [main] + extra, n // g
+    wg, wr = graphs(warmup)
+    w_ms = time_graphs(wg, wr, stream)
+    fg, fr = graphs(steps)
+    windows = int(min(50, max(1, np.ceil(500.0 / max(w_ms / warmup * steps, 1e-3)))))
+    uuid = str(torch.cuda.get_device_properties(device).uuid)
+    torch.cuda.synchronize(device)
+    with ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid) as clk:
+        ms_w = time_graphs(fg, fr, stream, windows)
+    ms_w = [ms_w] if windows == 1 else ms_w
+    ms = float(np.median(ms_w)) / steps
+    pk = peaks()
+    t_flops = flops / (pk["bf16"] * 1e12)
+    t_bytes = nbytes / (pk["hbm"] * 1e9)
+    if t_flops >= t_bytes:
+        roof = {"bound": "tensor", "achieved": flops / (ms / 1e3) / 1e12, "peak": pk["bf16"],
+                "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": nbytes / (ms / 1e3) / 1e9, "peak": pk["hbm"],
+                "unit": "GB/s"}
+    roof.update(frac=roof["achieved"] / roof["peak"], traffic=None, kernel="prep_gemm_kernel",
+                roofline_ms=max(t_flops, t_bytes) * 1e3,
+                peak_source=f"{pk['src']} (MEASURED_PEAKS.json)")
+    # the fp64 oracle on a bounded sample of tokens
+    rows = list(range(min(wl.T, 4)))
+    t0 = time.perf_counter()
+    sub = {k: (v[rows] if k in ("x", "qr", "cos", "sin") else v) for k, v in inputs.items()}
+    front_end(sub["x"], sub["qr"], sub["wq_b"], sub["wk"], sub["wp"], sub["gain"], sub["bias"],
+              sub["cos"], sub["sin"], H=wl.H, D=wl.D, rope_dim=wl.rope_dim, eps=1e-6,
+              w_scale=wl.w_scale)
+    dt = time.perf_counter() - t0
+    return {"metric": PREP_METRIC, "value": wl.T / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1,
+            "steps": steps, "warmup": warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "T": wl.T, "H": wl.H, "D": wl.D,
+                       "hidden": wl.hidden, "q_lora_rank": wl.q_lora_rank,
+                       "rope_dim": wl.rope_dim},
+            "timing": {"l2": f"{nsets} rotating input copies" if nsets > 1
+                       else "inputs larger than L2", "windows": windows,
+                       "ms_per_step_windows": [x / steps for x in ms_w]},
+            "tflops": flops / (ms / 1e3) / 1e12, "roofline": roof, "clocks": clk.summary(),
+            "cpu_baseline": {"value": len(rows) / dt, "unit": "tokens/s",
+                             "cores": os.cpu_count() or 1, "kind": "oracle",
+                             "sample": f"{len(rows)} of {wl.T} tokens (numpy fp64 matmuls), "
+                                       f"{dt:.2f} s"}}
+
+
 # ---------------------------------------------------------------- main
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
@@ -636,7 +745,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=None)
     ap.add_argument("--workload", default="ragged_prefill",
-                    choices=sorted(syn.WORKLOADS) + sorted(syn.MQA_WORKLOADS))
+                    choices=sorted(syn.WORKLOADS) + sorted(syn.MQA_WORKLOADS) +
+                    sorted(syn.PREPARE_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=None,
                     help="end-to-end steps (default 20; 5 for the ragged prefill)")
@@ -645,6 +755,17 @@ def main(argv=None):
                     help="packed causal workloads: other sequence lengths, comma "
                          "separated (a smaller batch of the same kind, for profiling)")
     args = ap.parse_args(argv)
+    if args.workload in syn.PREPARE_WORKLOADS:
+        wl = syn.PREPARE_WORKLOADS[args.workload]
+        d_steps, d_warm, _ = PREP_DEFAULTS[wl.name]
+        args.steps = d_steps if args.steps is None else args.steps
+        args.warmup = d_warm if args.warmup is None else args.warmup
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the oracle arm covers the "
+                              "indexer workloads only"}), flush=True)
+            return 0
+        print(json.dumps(run_prepare(args, wl)), flush=True)
+        return 0
     if args.workload in syn.MQA_WORKLOADS:
         wl = syn.MQA_WORKLOADS[args.workload]
         d_steps, d_warm, _ = MQA_DEFAULTS[wl.name]

@@ -340,3 +340,59 @@ def generate_mqa(wl: MqaWorkload, seed: Optional[int] = None) -> dict:
                 pick = rng.permutation(pick)[:m]
             idx[b, s, :m] = pick
     return dict(q=q, kv=kv, sinks=sinks, idx=idx)
+
+
+# ---- the indexer's front end: projections, LayerNorm, RoPE -------------------
+
+@dataclasses.dataclass(frozen=True)
+class PrepareWorkload:
+    """One synthetic front-end problem (DeepSeek-V3.2 Sparse Indexer Kernel API
+    Reference, Parameters). The pages fix head_dim = 128 and the 64-head
+    configuration; hidden, q_lora_rank and rope_dim take the published
+    DeepSeek-V3.2 sizes (7168, 1536, 64) unless stated."""
+    name: str
+    T: int
+    H: int = 64
+    hidden: int = 7168
+    q_lora_rank: int = 1536
+    rope_dim: int = 64
+    D: int = 128
+    seed: int = 0
+
+    @property
+    def w_scale(self) -> float:
+        return float(self.H * self.D) ** -0.5
+
+
+PREPARE_WORKLOADS = {
+    "prepare_decode": PrepareWorkload("prepare_decode", T=16),
+    "prepare_prefill": PrepareWorkload("prepare_prefill", T=8192),
+}
+
+
+def generate_prepare(wl: PrepareWorkload, seed: Optional[int] = None,
+                     positions: Optional[np.ndarray] = None) -> dict:
+    """Draw a front-end problem (host arrays; bf16 as bit patterns).
+
+    ``numpy.random.default_rng(seed)``, draws in the order x, qr, wq_b, wk,
+    weights_proj, gain, bias. Activations ~ N(0,1); weights ~ N(0,1) /
+    sqrt(in_features) (so projections are ~ N(0,1)); LayerNorm gain ~
+    1 + N(0,1)/10, bias ~ N(0,1)/10; cos/sin of the angles pos * 10000^(-2i /
+    rope_dim) at each token's position (positions t when not given)."""
+    rng = np.random.default_rng(wl.seed if seed is None else seed)
+    T, H, D, hid, ql = wl.T, wl.H, wl.D, wl.hidden, wl.q_lora_rank
+    x = f32_to_bf16_bits(gaussian_f32(rng, T * hid).reshape(T, hid))
+    qr = f32_to_bf16_bits(gaussian_f32(rng, T * ql).reshape(T, ql))
+    wq_b = f32_to_bf16_bits((gaussian_f32(rng, H * D * ql) / np.float32(np.sqrt(ql)))
+                            .reshape(H * D, ql))
+    wk = f32_to_bf16_bits((gaussian_f32(rng, D * hid) / np.float32(np.sqrt(hid))).reshape(D, hid))
+    wp = f32_to_bf16_bits((gaussian_f32(rng, H * hid) / np.float32(np.sqrt(hid))).reshape(H, hid))
+    gain = (1.0 + gaussian_f32(rng, D) / 10).astype(np.float32)
+    bias = (gaussian_f32(rng, D) / 10).astype(np.float32)
+    pos = np.arange(T, dtype=np.int32) if positions is None else np.asarray(positions, np.int32)
+    half = wl.rope_dim // 2
+    theta = 10000.0 ** (-2.0 * np.arange(half) / max(wl.rope_dim, 1))
+    ang = pos[:, None].astype(np.float64) * theta[None, :]
+    return dict(x=x, qr=qr, wq_b=wq_b, wk=wk, wp=wp, gain=gain, bias=bias,
+                cos=np.cos(ang).astype(np.float32), sin=np.sin(ang).astype(np.float32),
+                positions=pos)

@@ -36,7 +36,8 @@ DSA_FLAG_SELFTEST_STALL = 2
 EXPORTS = ("dsa_indexer_workspace_size", "dsa_indexer_score", "dsa_indexer_topk",
            "dsa_indexer_forward", "dsa_indexer_forward_noalloc",
            "dsa_indexer_get_error", "dsa_sparse_mqa_workspace_size",
-           "dsa_sparse_mqa_forward", "dsa_status_string")
+           "dsa_sparse_mqa_forward", "dsa_indexer_prepare_workspace_size",
+           "dsa_indexer_prepare", "dsa_status_string")
 
 
 class dsa_indexer_desc_t(ctypes.Structure):
@@ -56,6 +57,14 @@ class dsa_sparse_mqa_desc_t(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("S", ctypes.c_int32), ("H", ctypes.c_int32),
                 ("D", ctypes.c_int32), ("K", ctypes.c_int64), ("K_top", ctypes.c_int32),
                 ("sm_scale", ctypes.c_float), ("wait_limit_ns", ctypes.c_uint64)]
+
+
+class dsa_prepare_desc_t(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32), ("D", ctypes.c_int32),
+                ("hidden", ctypes.c_int32), ("q_lora_rank", ctypes.c_int32),
+                ("rope_dim", ctypes.c_int32), ("k_norm_eps", ctypes.c_float),
+                ("w_scale", ctypes.c_float), ("S", ctypes.c_int64),
+                ("k_seq_stride", ctypes.c_int64), ("wait_limit_ns", ctypes.c_uint64)]
 
 
 class DsaError(RuntimeError):
@@ -83,6 +92,9 @@ _lib.dsa_indexer_get_error.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_int)]
 _M = ctypes.POINTER(dsa_sparse_mqa_desc_t)
 _lib.dsa_sparse_mqa_workspace_size.argtypes = [_M, ctypes.POINTER(_sz)]
 _lib.dsa_sparse_mqa_forward.argtypes = [_M, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+_R = ctypes.POINTER(dsa_prepare_desc_t)
+_lib.dsa_indexer_prepare_workspace_size.argtypes = [_R, ctypes.POINTER(_sz)]
+_lib.dsa_indexer_prepare.argtypes = [_R] + [_vp] * 14 + [_sz, _vp]
 _lib.dsa_status_string.argtypes = [ctypes.c_int]
 _lib.dsa_status_string.restype = ctypes.c_char_p
 for _f in EXPORTS[:-1]:
@@ -207,3 +219,28 @@ def dsa_sparse_mqa_forward(desc, q, kv, sinks, topk, out, workspace, workspace_b
     return _check(_lib.dsa_sparse_mqa_forward(
         ctypes.byref(desc), _ptr(q), _ptr(kv), _ptr(sinks), _ptr(topk), _ptr(out),
         _ptr(workspace), workspace_bytes, stream), "dsa_sparse_mqa_forward")
+
+
+def make_prepare_desc(T, H, hidden, q_lora_rank, rope_dim, *, D=128, k_norm_eps=1e-6,
+                      w_scale=1.0, S=None, k_seq_stride=0, wait_limit_ns=0):
+    return dsa_prepare_desc_t(T=T, H=H, D=D, hidden=hidden, q_lora_rank=q_lora_rank,
+                              rope_dim=rope_dim, k_norm_eps=k_norm_eps, w_scale=w_scale,
+                              S=T if S is None else S, k_seq_stride=k_seq_stride,
+                              wait_limit_ns=wait_limit_ns)
+
+
+def dsa_indexer_prepare_workspace_size(desc) -> int:
+    n = _sz(0)
+    _check(_lib.dsa_indexer_prepare_workspace_size(ctypes.byref(desc), ctypes.byref(n)),
+           "dsa_indexer_prepare_workspace_size")
+    return n.value
+
+
+def dsa_indexer_prepare(desc, x, qr, wq_b, wk, weights_proj, k_norm_weight, k_norm_bias,
+                        cos, sin, positions, q_out, w_out, key_cache, workspace,
+                        workspace_bytes, stream=None) -> int:
+    return _check(_lib.dsa_indexer_prepare(
+        ctypes.byref(desc), _ptr(x), _ptr(qr), _ptr(wq_b), _ptr(wk), _ptr(weights_proj),
+        _ptr(k_norm_weight), _ptr(k_norm_bias), _ptr(cos), _ptr(sin), _ptr(positions),
+        _ptr(q_out), _ptr(w_out), _ptr(key_cache), _ptr(workspace), workspace_bytes,
+        stream), "dsa_indexer_prepare")

@@ -15,6 +15,7 @@
 #include "dsa_launch.h"
 #include "cu_check.cuh"
 #include "score_kernel.cuh"
+#include "topk_causal.cuh"
 #include "topk_cluster.cuh"
 #include "topk_rows.cuh"
 #include "topk_kernel.cuh"
@@ -427,7 +428,7 @@ dsa_status_t launch_score(const dsa_indexer_desc_t *d, const void *q, const uint
   if (launch_pdl(L.kernel, grid, L.threads(), plan.total, stream, 0, tk, tq, tksf, tqsf, p) !=
       cudaSuccess)
     return DSA_ERR_CUDA;
-  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+  return DSA_OK;
 }
 
 // The row top-k: one CTA per row, a buffer of NT*KPT floats.
@@ -436,7 +437,7 @@ dsa_status_t launch_topk_rows(DeviceInfo *dev, int which, int T, const TopkParam
                               cudaStream_t stream) {
   auto kernel = dsa::topk_rows_kernel<NT, KPT>;
   const int smem = NT * KPT * 4;
-  dsa_status_t st = ensure_smem_attr(dev, 16 + which, kernel, smem);
+  dsa_status_t st = ensure_smem_attr(dev, which ? kAttrTopkRows16 : kAttrTopkRows8, kernel, smem);
   if (st != DSA_OK) return st;
   if (launch_pdl(kernel, T, NT, smem, stream, 0, p) != cudaSuccess) return DSA_ERR_CUDA;
   return DSA_OK;
@@ -477,7 +478,7 @@ dsa_status_t launch_topk(const dsa_indexer_desc_t *d, const float *scores,
     const dsa_status_t rs = d->S + 3 <= 2048 ? launch_topk_rows<256, 8>(dev, 0, d->T, p, stream)
                                              : launch_topk_rows<256, 16>(dev, 1, d->T, p, stream);
     if (rs != DSA_OK) return rs;
-    return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+    return DSA_OK;
   }
   if (p.mode == dsa::kModePositions) {
     using Sh = dsa::ClusterTopkShared<512>;
@@ -487,21 +488,26 @@ dsa_status_t launch_topk(const dsa_indexer_desc_t *d, const float *scores,
     const int64_t room = (kMaxSmemPerBlock - sizeof(Sh) - 1024) / 4;
     p.stage_cap = static_cast<int>(std::min<int64_t>((d->S + C - 1) / C, room));
     const int smem = static_cast<int>(sizeof(Sh) + 4 * static_cast<size_t>(p.stage_cap));
-    st = ensure_smem_attr(dev, 8, dsa::topk_cluster_kernel<512>, static_cast<int>(kMaxSmemPerBlock));
+    st = ensure_smem_attr(dev, kAttrTopkCluster, dsa::topk_cluster_kernel<512>, static_cast<int>(kMaxSmemPerBlock));
     if (st != DSA_OK) return st;
     if (launch_pdl(dsa::topk_cluster_kernel<512>, d->T * C, 512, smem, stream, C, p) !=
         cudaSuccess)
       return DSA_ERR_CUDA;
   } else {
-    using Sh = dsa::TopkShared<512>;
-    p.stage_cap = std::min(d->T, 12288);
-    const int smem = static_cast<int>(sizeof(Sh) + 4 * static_cast<size_t>(p.stage_cap));
-    st = ensure_smem_attr(dev, 9, dsa::topk_kernel<512>, static_cast<int>(kMaxSmemPerBlock));
+    // packed causal rows: the two-pass kernel (its shared memory also holds
+    // the general selection's layout, which a crowded threshold bin falls
+    // back to)
+    p.stage_cap = 12288;
+    const size_t head = std::max((sizeof(dsa::CausalTopkShared<512>) + 15) & ~size_t(15),
+                                 sizeof(dsa::TopkShared<512>));
+    const int smem = static_cast<int>(head + 4 * static_cast<size_t>(p.stage_cap));
+    st = ensure_smem_attr(dev, kAttrTopkCausal, dsa::topk_causal_kernel<512>,
+                          static_cast<int>(kMaxSmemPerBlock));
     if (st != DSA_OK) return st;
-    if (launch_pdl(dsa::topk_kernel<512>, d->T, 512, smem, stream, 0, p) != cudaSuccess)
+    if (launch_pdl(dsa::topk_causal_kernel<512>, d->T, 512, smem, stream, 0, p) != cudaSuccess)
       return DSA_ERR_CUDA;
   }
-  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+  return DSA_OK;
 }
 
 dsa_status_t check_inputs(const dsa_indexer_desc_t *d, const void *q, const uint8_t *q_scale,

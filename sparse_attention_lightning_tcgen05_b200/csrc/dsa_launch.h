@@ -16,6 +16,18 @@ namespace dsa_host {
 
 constexpr size_t kWorkspaceHeader = 256;   // bytes of workspace every call needs
 
+// Bits of DeviceInfo::attr_done: one per kernel whose dynamic shared-memory
+// limit is raised (the score kernel's instances take 0 .. 15). Every kernel
+// needs its own bit: a shared one would skip another kernel's attribute.
+enum : uint32_t {
+  kAttrTopkRows8 = 16,
+  kAttrTopkRows16 = 17,
+  kAttrTopkCluster = 18,
+  kAttrTopkCausal = 19,
+  kAttrSparseMqa = 20,
+  kAttrPrepare = 21,
+};
+
 // What the library knows about a device (probed once per device).
 struct DeviceInfo {
   bool probed = false;
@@ -66,7 +78,11 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int threads, size_t s
     attr[1].val.clusterDim.z = 1;
     cfg.numAttrs = 2;
   }
-  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  // a launch this library failed is reported through its status: consume the
+  // error so that it is not mistaken for a later call's
+  if (e != cudaSuccess) (void)cudaGetLastError();
+  return e;
 }
 
 struct WsHeader;

@@ -89,7 +89,7 @@ dsa_status_t dsa_sparse_mqa_forward(const dsa_sparse_mqa_desc_t *desc, const voi
   st = device_info(&dev);
   if (st != DSA_OK) return st;
   const int smem = static_cast<int>(dsa::MqaSmem::total);
-  st = ensure_smem_attr(dev, 24, dsa::sparse_mqa_kernel, smem);
+  st = ensure_smem_attr(dev, kAttrSparseMqa, dsa::sparse_mqa_kernel, smem);
   if (st != DSA_OK) return st;
 
   const int T = desc->B * desc->S;
@@ -132,7 +132,7 @@ dsa_status_t dsa_sparse_mqa_forward(const dsa_sparse_mqa_desc_t *desc, const voi
   if (nsplit > 1 &&
       launch_pdl(dsa::sparse_mqa_combine_kernel, T, 256, 0, s, 0, p) != cudaSuccess)
     return DSA_ERR_CUDA;
-  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+  return DSA_OK;
 }
 
 }  // extern "C"

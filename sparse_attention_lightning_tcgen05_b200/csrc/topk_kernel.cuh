@@ -268,30 +268,13 @@ __device__ void stage_row(const float *row, uint32_t n, float *keys, TopkShared<
   block_minmax<NT>(lo, hi, sm);
 }
 
+// The selection of one row of n > k valid scores into out[0, k): the whole
+// block, smem `sm` and a stage of p.stage_cap floats. Every thread returns.
 template <int NT>
-__global__ void __launch_bounds__(NT) topk_kernel(const TopkParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  TopkShared<NT> &sm = *reinterpret_cast<TopkShared<NT> *>(smem_raw);
-  float *staged_keys = reinterpret_cast<float *>(smem_raw + sizeof(TopkShared<NT>));
-  const int t = blockIdx.x;
+__device__ void topk_row_full(const TopkParams &p, TopkShared<NT> &sm, float *staged_keys,
+                              const float *row, uint32_t n, int *out) {
   const int tid = threadIdx.x;
-  // scores (and positions) come from earlier work on the stream
-  grid_dep_wait();
-  grid_dep_launch_dependents();
-  // CAUSAL: a cu_seqlens array that failed its check -> write nothing
-  if (p.mode == kModeCausal && *p.cu_bad) return;
-
-  const float *row;
-  int64_t nvalid;
-  topk_row_geometry<NT>(p, t, sm, row, nvalid);
-  int *out = p.topk + static_cast<int64_t>(t) * p.k;
   const uint32_t k = static_cast<uint32_t>(p.k);
-
-  if (nvalid <= static_cast<int64_t>(k)) {
-    for (uint32_t i = tid; i < k; i += NT) out[i] = i < nvalid ? static_cast<int>(i) : -1;
-    return;
-  }
-  const uint32_t n = static_cast<uint32_t>(nvalid);
   const bool staged = n <= static_cast<uint32_t>(p.stage_cap);
 
   // ---- stage (or scan) the row: keys and their range ----
@@ -523,6 +506,32 @@ __global__ void __launch_bounds__(NT) topk_kernel(const TopkParams p) {
     base_gt += total >> 16;
     base_eq += total & 0xFFFFu;
   }
+}
+
+template <int NT>
+__global__ void __launch_bounds__(NT) topk_kernel(const TopkParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  TopkShared<NT> &sm = *reinterpret_cast<TopkShared<NT> *>(smem_raw);
+  float *staged_keys = reinterpret_cast<float *>(smem_raw + sizeof(TopkShared<NT>));
+  const int t = blockIdx.x;
+  const int tid = threadIdx.x;
+  // scores (and positions) come from earlier work on the stream
+  grid_dep_wait();
+  grid_dep_launch_dependents();
+  // CAUSAL: a cu_seqlens array that failed its check -> write nothing
+  if (p.mode == kModeCausal && *p.cu_bad) return;
+
+  const float *row;
+  int64_t nvalid;
+  topk_row_geometry<NT>(p, t, sm, row, nvalid);
+  int *out = p.topk + static_cast<int64_t>(t) * p.k;
+  const uint32_t k = static_cast<uint32_t>(p.k);
+
+  if (nvalid <= static_cast<int64_t>(k)) {
+    for (uint32_t i = tid; i < k; i += NT) out[i] = i < nvalid ? static_cast<int>(i) : -1;
+    return;
+  }
+  topk_row_full<NT>(p, sm, staged_keys, row, static_cast<uint32_t>(nvalid), out);
 }
 
 }  // namespace dsa

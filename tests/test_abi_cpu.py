@@ -360,3 +360,36 @@ def test_sparse_mqa_host_checks():
     with pytest.raises(dsa.DsaError) as e:               # workspace too small
         dsa.dsa_sparse_mqa_forward(d, fake, fake, fake, fake, fake, fake, 128)
     assert e.value.status == dsa.DSA_ERR_WORKSPACE
+
+
+def test_prepare_host_checks():
+    """The front end's descriptor and pointer checks run on the host; its
+    workspace is sized from the descriptor alone (the header, plus the fp32
+    partial rows of a projection whose K range is split)."""
+    d = dsa.make_prepare_desc(16, 64, 7168, 1536, 64)
+    n = dsa.dsa_indexer_prepare_workspace_size(d)
+    # queries: 64 tiles, 3 splits of 8 K steps -> 3 x 16 x 8192 floats;
+    # keys + weights: 1 tile, 28 splits -> 28 x 16 x 192 floats
+    assert n == 256 + max(3 * 16 * 8192 * 4, 28 * 16 * 192 * 4)
+    assert dsa.dsa_indexer_prepare_workspace_size(dsa.make_prepare_desc(300, 64, 256, 256, 64)) == 256
+    for kw, code in ((dict(H=24), dsa.DSA_ERR_UNSUPPORTED), (dict(H=144), dsa.DSA_ERR_UNSUPPORTED),
+                     (dict(D=64), dsa.DSA_ERR_UNSUPPORTED), (dict(hidden=100), dsa.DSA_ERR_UNSUPPORTED),
+                     (dict(rope_dim=63), dsa.DSA_ERR_INVALID_ARG),
+                     (dict(rope_dim=130), dsa.DSA_ERR_INVALID_ARG),
+                     (dict(k_norm_eps=-1.0), dsa.DSA_ERR_INVALID_ARG),
+                     (dict(k_seq_stride=1000), dsa.DSA_ERR_INVALID_ARG)):
+        args = dict(T=4, H=64, hidden=256, q_lora_rank=256, rope_dim=64)
+        args.update(kw)
+        with pytest.raises(dsa.DsaError) as e:
+            dsa.dsa_indexer_prepare_workspace_size(dsa.make_prepare_desc(**args))
+        assert e.value.status == code
+    fake = 1 << 20
+    d = dsa.make_prepare_desc(4, 64, 256, 256, 64)
+    args = [fake] * 13                                  # x .. key_cache
+    args[0] = fake + 2                                   # misaligned x
+    with pytest.raises(dsa.DsaError) as e:
+        dsa.dsa_indexer_prepare(d, *args, fake, 256)
+    assert e.value.status == dsa.DSA_ERR_INVALID_ARG
+    with pytest.raises(dsa.DsaError) as e:               # workspace too small
+        dsa.dsa_indexer_prepare(d, *([fake] * 13), fake, 64)
+    assert e.value.status == dsa.DSA_ERR_WORKSPACE

@@ -31,6 +31,17 @@ constexpr uint64_t kDrainLimitNs = 4000000000ull;  // drains of in-flight copies
 constexpr int kMaxDevices = 64;
 constexpr uint32_t kMaxSmemPerBlock = 232448;      // 227 KB opt-in limit of sm_100
 
+// Packed causal top-k: threads per row and scores staged in shared memory
+// (longer rows stream from L2 in their second pass). Build-time tunables.
+#ifndef DSA_CAUSAL_TOPK_THREADS
+#define DSA_CAUSAL_TOPK_THREADS 512
+#endif
+#ifndef DSA_CAUSAL_TOPK_STAGE
+#define DSA_CAUSAL_TOPK_STAGE 12288
+#endif
+constexpr int kCausalTopkThreads = DSA_CAUSAL_TOPK_THREADS;
+constexpr int kCausalTopkStage = DSA_CAUSAL_TOPK_STAGE;
+
 // Words of the workspace header.
 // err/err_info: first device-side failure since the last get_error (sticky).
 // cu_bad: written by the cu_seqlens check of every CAUSAL call, read by that
@@ -497,14 +508,15 @@ dsa_status_t launch_topk(const dsa_indexer_desc_t *d, const float *scores,
     // packed causal rows: the two-pass kernel (its shared memory also holds
     // the general selection's layout, which a crowded threshold bin falls
     // back to)
-    p.stage_cap = 12288;
-    const size_t head = std::max((sizeof(dsa::CausalTopkShared<512>) + 15) & ~size_t(15),
-                                 sizeof(dsa::TopkShared<512>));
+    constexpr int NT = kCausalTopkThreads;
+    p.stage_cap = kCausalTopkStage;
+    const size_t head = std::max((sizeof(dsa::CausalTopkShared<NT>) + 15) & ~size_t(15),
+                                 sizeof(dsa::TopkShared<NT>));
     const int smem = static_cast<int>(head + 4 * static_cast<size_t>(p.stage_cap));
-    st = ensure_smem_attr(dev, kAttrTopkCausal, dsa::topk_causal_kernel<512>,
+    st = ensure_smem_attr(dev, kAttrTopkCausal, dsa::topk_causal_kernel<NT>,
                           static_cast<int>(kMaxSmemPerBlock));
     if (st != DSA_OK) return st;
-    if (launch_pdl(dsa::topk_causal_kernel<512>, d->T, 512, smem, stream, 0, p) != cudaSuccess)
+    if (launch_pdl(dsa::topk_causal_kernel<NT>, d->T, NT, smem, stream, 0, p) != cudaSuccess)
       return DSA_ERR_CUDA;
   }
   return DSA_OK;

@@ -40,17 +40,29 @@ struct Split {
   int m_tiles, n_tiles, ksteps, nsplit, per;
 };
 
+// K splits: the count that minimises (waves of items over the SMs) x (K steps
+// an item runs + the fixed cost of an item, about 3 K steps), at most 32
+// splits (the reduction sums them).
 Split plan(int T, int n_tiles, int K) {
   Split s{};
   s.m_tiles = (T + 127) / 128;
   s.n_tiles = n_tiles;
   s.ksteps = K / dsa::kPrepBK;
-  const int items = s.m_tiles * n_tiles;
-  int want = 1;
-  if (items < kSizingSms) want = (kSizingSms + items - 1) / items;
-  want = std::max(1, std::min(want, s.ksteps / 4));
-  s.per = (s.ksteps + want - 1) / want;
-  s.nsplit = (s.ksteps + s.per - 1) / s.per;
+  const int64_t tiles = static_cast<int64_t>(s.m_tiles) * n_tiles;
+  int64_t best = -1;
+  s.nsplit = 1;
+  s.per = s.ksteps;
+  for (int want = 1; want <= std::min(32, s.ksteps); ++want) {
+    const int per = (s.ksteps + want - 1) / want;
+    const int ns = (s.ksteps + per - 1) / per;
+    const int64_t waves = (tiles * ns + kSizingSms - 1) / kSizingSms;
+    const int64_t cost = waves * (per + 3);
+    if (best < 0 || cost < best) {
+      best = cost;
+      s.nsplit = ns;
+      s.per = per;
+    }
+  }
   return s;
 }
 
@@ -81,9 +93,12 @@ dsa_status_t launch_gemm(DeviceInfo *dev, const CUtensorMap &a, const CUtensorMa
                  static_cast<size_t>(dsa::PrepSmem::total), s, 0, a, b1, b2, p) != cudaSuccess)
     return DSA_ERR_CUDA;
   if (p.nsplit > 1) {
-    const int64_t warps = static_cast<int64_t>(p.T) * p.n_tiles;
-    const int blocks = static_cast<int>((warps * 32 + 255) / 256);
-    if (launch_pdl(dsa::prep_reduce_kernel, blocks, 256, 0, s, 0, p) != cudaSuccess)
+    // one CTA per (token, feature tile); up to 4 thread groups a column share
+    // the splits
+    const int bnp = (p.BN + 31) & ~31;
+    const int groups = std::max(1, std::min({4, (p.nsplit + 7) / 8, 1024 / bnp}));
+    if (launch_pdl(dsa::prep_reduce_kernel, p.T * p.n_tiles, groups * bnp, 0, s, 0, p,
+                   groups) != cudaSuccess)
       return DSA_ERR_CUDA;
   }
   return DSA_OK;

@@ -129,9 +129,12 @@ dsa_status_t dsa_sparse_mqa_forward(const dsa_sparse_mqa_desc_t *desc, const voi
   if (launch_pdl(dsa::sparse_mqa_kernel, grid, dsa::kMqaThreads, static_cast<size_t>(smem), s, 0,
                  tq, p) != cudaSuccess)
     return DSA_ERR_CUDA;
-  if (nsplit > 1 &&
-      launch_pdl(dsa::sparse_mqa_combine_kernel, T, 256, 0, s, 0, p) != cudaSuccess)
-    return DSA_ERR_CUDA;
+  if (nsplit > 1) {
+    const int64_t warps = static_cast<int64_t>(T) * desc->H;   // one per (token, head)
+    const int blocks = static_cast<int>((warps * 32 + 255) / 256);
+    if (launch_pdl(dsa::sparse_mqa_combine_kernel, blocks, 256, 0, s, 0, p) != cudaSuccess)
+      return DSA_ERR_CUDA;
+  }
   return DSA_OK;
 }
 

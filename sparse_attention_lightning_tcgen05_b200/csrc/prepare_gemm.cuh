@@ -350,57 +350,84 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
-// Sum of the K splits and the epilogue: one warp per (token, feature tile);
-// lane l holds columns 4l .. 4l+3 of the tile's first 128 (and, in mode KW,
-// head weights l, l + 32, ...).
-__global__ void __launch_bounds__(256) prep_reduce_kernel(const PrepParams p) {
+// Sum of the K splits and the epilogue. One CTA per (token, feature tile);
+// column c of the tile belongs to threads c + g * BNp (g < groups, BNp = BN
+// rounded up to a warp): group g sums the splits g, g + groups, ... with four
+// loads in flight, and group 0 adds the groups' sums. Then, for the columns:
+//   mode Q : RoPE (the pair partner is the neighbouring lane), bf16 q;
+//   mode KW: LayerNorm over the key's 128 columns (block reduction), RoPE,
+//            the bf16 key row into the cache; the H head weights scaled.
+__global__ void __launch_bounds__(1024) prep_reduce_kernel(const PrepParams p, int groups) {
+  __shared__ float part_sum[1024];
+  __shared__ float red[2][4];
   grid_dep_wait();
   grid_dep_launch_dependents();
-  const int lane = threadIdx.x & 31;
-  const int64_t wid = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwork = static_cast<int64_t>(p.T) * p.n_tiles;
-  if (wid >= nwork) return;
-  const int t = static_cast<int>(wid / p.n_tiles), nt = static_cast<int>(wid % p.n_tiles);
-  auto col_sum = [&](int c) {
-    float s = 0.f;
-    for (int sp = 0; sp < p.nsplit; ++sp)
-      s += p.part[(static_cast<int64_t>(sp) * p.T + t) * p.N_total + nt * p.BN + c];
-    return s;
-  };
-  float v[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) v[j] = col_sum(4 * lane + j);
+  const int BNp = (p.BN + 31) & ~31;
+  const int g = threadIdx.x / BNp, c = threadIdx.x % BNp;
+  const int t = blockIdx.x / p.n_tiles, nt = blockIdx.x % p.n_tiles;
+  float v = 0.f;
+  if (c < p.BN && g < groups) {
+    const float *src = p.part + static_cast<int64_t>(t) * p.N_total + nt * p.BN + c;
+    const int64_t step = static_cast<int64_t>(p.T) * p.N_total;
+    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+    int sp = g;
+    for (; sp + 3 * groups < p.nsplit; sp += 4 * groups) {
+      s0 += src[sp * step];
+      s1 += src[(sp + groups) * step];
+      s2 += src[(sp + 2 * groups) * step];
+      s3 += src[(sp + 3 * groups) * step];
+    }
+    for (; sp < p.nsplit; sp += groups) s0 += src[sp * step];
+    v = (s0 + s1) + (s2 + s3);
+  }
+  part_sum[threadIdx.x] = v;
+  __syncthreads();
+  if (g != 0) return;
+  for (int k = 1; k < groups; ++k) v += part_sum[k * BNp + c];
   const float *cosr = p.cos + static_cast<int64_t>(t) * (p.rope_dim / 2);
   const float *sinr = p.sin + static_cast<int64_t>(t) * (p.rope_dim / 2);
-  if (p.mode == kPrepQ) {
-    rope_chunk(v, 4 * lane, p.rope_dim, cosr, sinr);
-    uint2 *dst = reinterpret_cast<uint2 *>(p.q_out + (static_cast<int64_t>(t) * p.H + nt) * kPrepD);
-    dst[lane] = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+  const int warp = c >> 5, lane = c & 31;
+  // RoPE of the column pair (c & ~1, c | 1): the partner is the next lane over
+  auto rope1 = [&](float x) {
+    const float other = __shfl_xor_sync(0xffffffffu, x, 1);
+    if (c >= p.rope_dim) return x;
+    const float cs = __ldg(cosr + c / 2), sn = __ldg(sinr + c / 2);
+    return (c & 1) ? other * sn + x * cs : x * cs - other * sn;
+  };
+  if (p.mode == kPrepQ) {                      // 128 columns, four full warps
+    const float y = rope1(v);
+    const __nv_bfloat16 b = __float2bfloat16_rn(y);
+    p.q_out[(static_cast<int64_t>(t) * p.H + nt) * kPrepD + c] =
+        *reinterpret_cast<const uint16_t *>(&b);
     return;
   }
-  float s = v[0] + v[1] + v[2] + v[3];
+  if (warp < kPrepD / 32) {                    // the key: warps 0..3
+    float s = v;
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  const float mean = s * (1.f / kPrepD);
-  float q = 0.f;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    v[j] -= mean;
-    q += v[j] * v[j];
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (lane == 0) red[0][warp] = s;
   }
+  __syncthreads();
+  const float mean = (red[0][0] + red[0][1] + red[0][2] + red[0][3]) * (1.f / kPrepD);
+  if (warp < kPrepD / 32) {
+    const float d = v - mean;
+    float q = d * d;
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) q += __shfl_xor_sync(0xffffffffu, q, off);
-  const float rstd = rsqrtf(q * (1.f / kPrepD) + p.eps);
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-    v[j] = v[j] * rstd * __ldg(p.gain + 4 * lane + j) + __ldg(p.bias + 4 * lane + j);
-  rope_chunk(v, 4 * lane, p.rope_dim, cosr, sinr);
-  uint16_t *krow = prep_key_row(p, t);
-  if (krow)
-    reinterpret_cast<uint2 *>(krow)[lane] =
-        make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
-  for (int c = lane; c < p.H; c += 32)
-    p.w_out[static_cast<int64_t>(t) * p.H + c] = col_sum(kPrepD + c) * p.w_scale;
+    for (int off = 16; off > 0; off >>= 1) q += __shfl_xor_sync(0xffffffffu, q, off);
+    if (lane == 0) red[1][warp] = q;
+  }
+  __syncthreads();
+  if (warp < kPrepD / 32) {
+    const float var = (red[1][0] + red[1][1] + red[1][2] + red[1][3]) * (1.f / kPrepD);
+    const float y = rope1((v - mean) * rsqrtf(var + p.eps) * __ldg(p.gain + c) + __ldg(p.bias + c));
+    uint16_t *krow = prep_key_row(p, t);
+    if (krow) {
+      const __nv_bfloat16 b = __float2bfloat16_rn(y);
+      krow[c] = *reinterpret_cast<const uint16_t *>(&b);
+    }
+  } else if (c < kPrepD + p.H) {
+    p.w_out[static_cast<int64_t>(t) * p.H + (c - kPrepD)] = v * p.w_scale;
+  }
 }
 
 }  // namespace dsa

@@ -439,42 +439,59 @@ __global__ void __launch_bounds__(kMqaThreads, 1)
 
 // Merge of the nsplit ranges of each token: with M the largest range max,
 //   out = sum_c 2^(m_c - M) O_c / (sum_c 2^(m_c - M) l_c + 2^(sink - M)),
-// and out = 0 when no range kept an entry. One CTA per token.
+// and out = 0 when no range kept an entry. One warp per (token, head): lane
+// l merges columns 4l .. 4l+3; the ranges' (max, sum) pairs are read by the
+// first nsplit lanes and shared by shuffles.
 __global__ void __launch_bounds__(256) sparse_mqa_combine_kernel(const MqaParams p) {
   grid_dep_wait();
   grid_dep_launch_dependents();
-  const int t = blockIdx.x;
-  const int H = p.H;
+  const int lane = threadIdx.x & 31;
+  const int64_t wid = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (wid >= static_cast<int64_t>(p.T) * p.H) return;
+  const int t = static_cast<int>(wid / p.H), h = static_cast<int>(wid % p.H);
   const float neg_inf = -__int_as_float(0x7f800000);
-  for (int i = threadIdx.x; i < H * (kMqaD / 4); i += blockDim.x) {
-    const int h = i / (kMqaD / 4), d4 = i - h * (kMqaD / 4);
-    const float2 *ml = reinterpret_cast<const float2 *>(p.part_ml) +
-                       static_cast<int64_t>(t) * p.nsplit * H + h;
-    float M = neg_inf;
-    for (int c = 0; c < p.nsplit; ++c) M = fmaxf(M, ml[static_cast<int64_t>(c) * H].x);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float L = 0.f;
-    if (M != neg_inf) {
-      for (int c = 0; c < p.nsplit; ++c) {
-        const float2 v = ml[static_cast<int64_t>(c) * H];
-        const float w = v.x == neg_inf ? 0.f : ex2_approx(v.x - M);
-        L += w * v.y;
+  const float2 *ml = reinterpret_cast<const float2 *>(p.part_ml) +
+                     static_cast<int64_t>(t) * p.nsplit * p.H + h;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float L = 0.f, M = neg_inf;
+  for (int c0 = 0; c0 < p.nsplit; c0 += 32) {      // the ranges' maxima
+    const int c = c0 + lane;
+    const float m = c < p.nsplit ? ml[static_cast<int64_t>(c) * p.H].x : neg_inf;
+    M = fmaxf(M, m);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  if (M != neg_inf) {
+    for (int c0 = 0; c0 < p.nsplit; c0 += 32) {
+      const int c = c0 + lane;
+      float w = 0.f, l = 0.f;
+      if (c < p.nsplit) {
+        const float2 v = ml[static_cast<int64_t>(c) * p.H];
+        w = v.x == neg_inf ? 0.f : ex2_approx(v.x - M);
+        l = v.y;
+      }
+      L += w * l;
+      const int n = min(32, p.nsplit - c0);
+      for (int j = 0; j < n; ++j) {
+        const float wj = __shfl_sync(0xffffffffu, w, j);
         const float4 o = reinterpret_cast<const float4 *>(
-            p.part_o + ((static_cast<int64_t>(t) * p.nsplit + c) * H + h) * kMqaD)[d4];
-        acc.x += w * o.x;
-        acc.y += w * o.y;
-        acc.z += w * o.z;
-        acc.w += w * o.w;
+            p.part_o + ((static_cast<int64_t>(t) * p.nsplit + c0 + j) * p.H + h) * kMqaD)[lane];
+        acc.x += wj * o.x;
+        acc.y += wj * o.y;
+        acc.z += wj * o.z;
+        acc.w += wj * o.w;
       }
     }
-    const float inv = L > 0.f ? 1.f / (L + ex2_approx(__ldg(p.sinks + h) * kLog2e - M)) : 0.f;
-    const __nv_bfloat162 a = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-    const __nv_bfloat162 b = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-    uint2 w2;
-    w2.x = *reinterpret_cast<const uint32_t *>(&a);
-    w2.y = *reinterpret_cast<const uint32_t *>(&b);
-    reinterpret_cast<uint2 *>(p.out + (static_cast<int64_t>(t) * H + h) * kMqaD)[d4] = w2;
   }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+  const float inv = L > 0.f ? 1.f / (L + ex2_approx(__ldg(p.sinks + h) * kLog2e - M)) : 0.f;
+  const __nv_bfloat162 a = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+  const __nv_bfloat162 b = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+  uint2 w2;
+  w2.x = *reinterpret_cast<const uint32_t *>(&a);
+  w2.y = *reinterpret_cast<const uint32_t *>(&b);
+  reinterpret_cast<uint2 *>(p.out + (static_cast<int64_t>(t) * p.H + h) * kMqaD)[lane] = w2;
 }
 
 }  // namespace dsa

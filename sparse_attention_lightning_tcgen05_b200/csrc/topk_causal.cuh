@@ -188,7 +188,10 @@ __global__ void __launch_bounds__(NT) topk_causal_kernel(const TopkParams p) {
         eq |= static_cast<uint32_t>((valid >> q & 1u) && d == b1) << q;
       }
       warp_append4(gt, s0, &sm.nout, out, k);
-      warp_append4_cand(eq, s0, kk, &sm.ncand, sm.ckey, sm.cslot);
+      // members of the threshold bin are a few percent of the row: most
+      // rounds have none in the whole warp
+      if (__any_sync(0xffffffffu, eq != 0u))
+        warp_append4_cand(eq, s0, kk, &sm.ncand, sm.ckey, sm.cslot);
     };
     // head and tail slots: one per thread, as a 1-slot group
     const uint32_t edge = head + (n - tail0);

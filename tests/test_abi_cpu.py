@@ -368,10 +368,14 @@ def test_prepare_host_checks():
     partial rows of a projection whose K range is split)."""
     d = dsa.make_prepare_desc(16, 64, 7168, 1536, 64)
     n = dsa.dsa_indexer_prepare_workspace_size(d)
-    # queries: 64 tiles, 3 splits of 8 K steps -> 3 x 16 x 8192 floats;
-    # keys + weights: 1 tile, 28 splits -> 28 x 16 x 192 floats
-    assert n == 256 + max(3 * 16 * 8192 * 4, 28 * 16 * 192 * 4)
-    assert dsa.dsa_indexer_prepare_workspace_size(dsa.make_prepare_desc(300, 64, 256, 256, 64)) == 256
+    # queries: 64 tiles, 2 splits of 12 K steps -> 2 x 16 x 8192 floats (one
+    # wave of 128 items); keys + weights: 1 tile, 28 splits of 4 K steps ->
+    # 28 x 16 x 192 floats
+    assert n == 256 + max(2 * 16 * 8192 * 4, 28 * 16 * 192 * 4)
+    # 300 tokens, K = 256: 3 x 64 query tiles fill the SMs, the key tile
+    # splits its 4 K steps in 4
+    assert dsa.dsa_indexer_prepare_workspace_size(dsa.make_prepare_desc(300, 64, 256, 256, 64)) == \
+        256 + 4 * 300 * 192 * 4
     for kw, code in ((dict(H=24), dsa.DSA_ERR_UNSUPPORTED), (dict(H=144), dsa.DSA_ERR_UNSUPPORTED),
                      (dict(D=64), dsa.DSA_ERR_UNSUPPORTED), (dict(hidden=100), dsa.DSA_ERR_UNSUPPORTED),
                      (dict(rope_dim=63), dsa.DSA_ERR_INVALID_ARG),

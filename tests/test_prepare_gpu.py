@@ -97,16 +97,36 @@ def test_prepare_decode_split_k(dsa):
 
 
 @pytest.mark.parametrize("H,rope_dim", [(64, 64), (16, 0), (32, 128), (128, 64)])
-def test_prepare_fused_epilogues(dsa, H, rope_dim):
-    """Short contractions (hidden = q_lora_rank = 256): no K split, the
-    epilogues run in the GEMM kernel; 300 tokens (three token tiles, a
-    ragged last one), keys packed at slot t (prefill)."""
+def test_prepare_short_contractions(dsa, H, rope_dim):
+    """hidden = q_lora_rank = 256, 300 tokens (three token tiles, a ragged
+    last one), keys packed at slot t (prefill): the query GEMM runs unsplit
+    with its epilogue fused, the key/weight GEMM splits its four K steps."""
     wl = syn.PrepareWorkload("p", T=300, H=H, hidden=256, q_lora_rank=256, rope_dim=rope_dim,
                              seed=H + rope_dim)
     inp = syn.generate_prepare(wl)
     q, w, cache, nbytes = run(dsa, wl, inp)
-    assert nbytes == 256
+    assert nbytes > 256
     check(wl, inp, q, w, cache, [(t, t) for t in range(wl.T)])
+
+
+@pytest.mark.parametrize("H,rope_dim", [(64, 64), (16, 0)])
+def test_prepare_fused_epilogues(dsa, H, rope_dim):
+    """19000 tokens (149 token tiles) with K = 256: both GEMMs fill the SMs
+    unsplit, so the LayerNorm / RoPE / cache-write and the head-weight
+    epilogues run inside the GEMM kernel. Sampled rows."""
+    wl = syn.PrepareWorkload("pf", T=19000, H=H, hidden=256, q_lora_rank=256,
+                             rope_dim=rope_dim, seed=7 + H)
+    inp = syn.generate_prepare(wl)
+    q, w, cache, nbytes = run(dsa, wl, inp)
+    assert nbytes == 256
+    rows = [0, 1, 127, 128, 9000, 18943, 18944, 18999]
+    sub = {k: (v[rows] if k in ("x", "qr", "cos", "sin", "positions") else v)
+           for k, v in inp.items()}
+    oq, ok, ow = oracle(wl, sub)
+    close_bf16(q[rows], oq)
+    close_w(w[rows], ow)
+    for i, t in enumerate(rows):
+        close_bf16(bf16_to_f64(cache[t]), ok[i])
 
 
 def test_prepare_prefill_sizes(dsa):
@@ -116,11 +136,13 @@ def test_prepare_prefill_sizes(dsa):
     inp = syn.generate_prepare(wl)
     q, w, cache, _ = run(dsa, wl, inp)
     rows = [0, 1, 127, 128, 1000, 2047]
-    oq, ok, ow = oracle(wl, inp)
-    close_bf16(q[rows], oq[rows])
-    close_w(w[rows], ow[rows])
-    for t in rows:
-        close_bf16(bf16_to_f64(cache[t]), ok[t])
+    sub = {k: (v[rows] if k in ("x", "qr", "cos", "sin", "positions") else v)
+           for k, v in inp.items()}
+    oq, ok, ow = oracle(wl, sub)
+    close_bf16(q[rows], oq)
+    close_w(w[rows], ow)
+    for i, t in enumerate(rows):
+        close_bf16(bf16_to_f64(cache[t]), ok[i])
 
 
 def test_prepare_positions_outside_the_cache_write_nothing(dsa):

@@ -31,8 +31,9 @@ constexpr uint64_t kDrainLimitNs = 4000000000ull;  // drains of in-flight copies
 constexpr int kMaxDevices = 64;
 constexpr uint32_t kMaxSmemPerBlock = 232448;      // 227 KB opt-in limit of sm_100
 
-// Packed causal top-k: threads per row and scores staged in shared memory
-// (longer rows stream from L2 in their second pass). Build-time tunables.
+// Packed causal top-k: threads per row, and the scores a row may stage in
+// shared memory (rows that fit take the two-pass selection, longer rows the
+// sampled threshold). Build-time tunables.
 #ifndef DSA_CAUSAL_TOPK_THREADS
 #define DSA_CAUSAL_TOPK_THREADS 512
 #endif
@@ -510,9 +511,12 @@ dsa_status_t launch_topk(const dsa_indexer_desc_t *d, const float *scores,
     // back to)
     constexpr int NT = kCausalTopkThreads;
     p.stage_cap = kCausalTopkStage;
-    const size_t head = std::max((sizeof(dsa::CausalTopkShared<NT>) + 15) & ~size_t(15),
-                                 sizeof(dsa::TopkShared<NT>));
-    const int smem = static_cast<int>(head + 4 * static_cast<size_t>(p.stage_cap));
+    // the largest of the three layouts: the two-pass selection's and the
+    // general one's (each with the stage), the sampled threshold's
+    const size_t stage = 4 * static_cast<size_t>(p.stage_cap);
+    const int smem = static_cast<int>(
+        std::max({((sizeof(dsa::TwoPassShared<NT>) + 15) & ~size_t(15)) + stage,
+                  sizeof(dsa::TopkShared<NT>) + stage, sizeof(dsa::SampledShared<NT>)}));
     st = ensure_smem_attr(dev, kAttrTopkCausal, dsa::topk_causal_kernel<NT>,
                           static_cast<int>(kMaxSmemPerBlock));
     if (st != DSA_OK) return st;

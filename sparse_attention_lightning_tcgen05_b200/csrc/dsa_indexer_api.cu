@@ -478,17 +478,20 @@ dsa_status_t launch_topk(const dsa_indexer_desc_t *d, const float *scores,
   p.scores = scores;
   p.topk = topk;
   p.k = d->index_topk;
-  // Decode-style rows of at most 4093 slots (pooled keys, short caches): one
+  // Decode-style rows of at most 4096 slots (pooled keys, short caches): one
   // CTA a row, the row held in registers. A row's buffer starts at the
-  // 16-byte boundary at or before it, up to 3 floats early, so an instance
-  // holding NT*KPT floats takes rows of up to NT*KPT - 3 slots. Longer decode
-  // rows are few and long: a cluster of C CTAs per row (up to 8, about 4096
-  // slots each), the row staged across their shared memories. Prefill rows
-  // are many: 512 threads a row and a smaller stage, so that several rows run
-  // on each SM.
-  if (p.mode == dsa::kModePositions && d->S + 3 <= 4096) {
-    const dsa_status_t rs = d->S + 3 <= 2048 ? launch_topk_rows<256, 8>(dev, 0, d->T, p, stream)
-                                             : launch_topk_rows<256, 16>(dev, 1, d->T, p, stream);
+  // 16-byte boundary at or before it, up to 3 floats early (none when the
+  // score buffer is 16-byte aligned and S a multiple of 4), so an instance
+  // holding NT*KPT floats takes rows of up to NT*KPT - 3 slots (NT*KPT when
+  // every row is aligned). Longer decode rows are few and long: a cluster of
+  // C CTAs per row (up to 8, about 4096 slots each), the row staged across
+  // their shared memories. Prefill rows are many: 512 threads a row and a
+  // smaller stage, so that several rows run on each SM.
+  const int64_t lead = (aligned(scores, 16) && d->S % 4 == 0) ? 0 : 3;
+  if (p.mode == dsa::kModePositions && d->S + lead <= 4096) {
+    const dsa_status_t rs = d->S + lead <= 2048
+                                ? launch_topk_rows<256, 8>(dev, 0, d->T, p, stream)
+                                : launch_topk_rows<256, 16>(dev, 1, d->T, p, stream);
     if (rs != DSA_OK) return rs;
     return DSA_OK;
   }

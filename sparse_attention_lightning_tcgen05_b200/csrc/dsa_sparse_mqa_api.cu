@@ -29,7 +29,8 @@ dsa_status_t check_mqa_desc(const dsa_sparse_mqa_desc_t *d) {
   if (d->D != 128) return DSA_ERR_UNSUPPORTED;
   if (d->H > 128) return DSA_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(d->B) * d->S * d->H > INT32_MAX - 256) return DSA_ERR_UNSUPPORTED;
-  if (d->K > INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  // kv rows are addressed as 32-bit TMA coordinates over all batches
+  if (static_cast<int64_t>(d->B) * d->K >= INT32_MAX) return DSA_ERR_UNSUPPORTED;
   return DSA_OK;
 }
 
@@ -101,6 +102,15 @@ dsa_status_t dsa_sparse_mqa_forward(const dsa_sparse_mqa_desc_t *desc, const voi
     st = make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, dims, strides, box);
     if (st != DSA_OK) return st;
   }
+  // the kv rows of all batches, one row a box (tile::gather4 loads four)
+  CUtensorMap tkv;
+  {
+    const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(desc->B) * desc->K};
+    const cuuint64_t strides[1] = {256};
+    const cuuint32_t box[2] = {64, 1};
+    st = make_map(&tkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kv, dims, strides, box);
+    if (st != DSA_OK) return st;
+  }
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   dsa::MqaParams p{};
   p.T = T;
@@ -127,7 +137,7 @@ dsa_status_t dsa_sparse_mqa_forward(const dsa_sparse_mqa_desc_t *desc, const voi
   const int grid = static_cast<int>(std::min<int64_t>(items, dev->num_sms));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (launch_pdl(dsa::sparse_mqa_kernel, grid, dsa::kMqaThreads, static_cast<size_t>(smem), s, 0,
-                 tq, p) != cudaSuccess)
+                 tq, tkv, p) != cudaSuccess)
     return DSA_ERR_CUDA;
   if (nsplit > 1) {
     const int64_t warps = static_cast<int64_t>(T) * desc->H;   // one per (token, head)

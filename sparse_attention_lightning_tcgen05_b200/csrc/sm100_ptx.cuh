@@ -573,3 +573,22 @@ __device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t *bar) {
 }
 
 }  // namespace dsa
+
+namespace dsa {
+
+// Four rows (y0..y3) of a 2D tensor whose map has a one-row box, into four
+// consecutive box rows of shared memory at dst (the map's swizzle applied by
+// address; dst aligned like the whole four-row block). A row coordinate
+// outside the tensor reads as zeros; the mbarrier counts the full bytes.
+__device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *map, uint64_t *bar,
+                                            int32_t x, int32_t y0, int32_t y1, int32_t y2,
+                                            int32_t y3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1),
+      "r"(y2), "r"(y3)
+      : "memory");
+}
+
+}  // namespace dsa

@@ -16,10 +16,12 @@
 // it, or 1/nsplit of it when there are too few tokens to fill the GPU; a
 // second kernel then merges the ranges). Persistent CTAs, one per SM, walk
 // the items. Per tile of 128 index entries:
-//   producer warps 5, 6 : each thread gathers two selected kv rows (256 bytes
-//                         each) with 16-byte cp.async copies into a 128-byte-
-//                         swizzled K-major tile (masked rows: zero-filled) and
-//                         publishes the tile's validity bits;
+//   producer warp 5     : lane l gathers the tile's rows 4l .. 4l+3 with TMA
+//                         tile::gather4 loads (four 128-byte row halves an
+//                         instruction, two a lane) into a 128-byte-swizzled
+//                         K-major tile; a masked entry reads a row past the
+//                         tensor, which TMA fills with zeros; lane 0 publishes
+//                         the tile's validity bits;
 //   MMA warp 4          : S = Q K^T  (M = 128 head rows, N = 128 keys, K = D)
 //                         into one of two TMEM score buffers, then
 //                         O += P V    (M = 128 head rows, N = D, K = 128 keys)
@@ -44,9 +46,9 @@ constexpr int kMqaD = 128;               // head dim (the indexer's)
 constexpr int kMqaTile = 128;            // index entries per tile
 constexpr int kMqaStages = 3;            // gathered kv tiles in flight
 constexpr int kMqaSoftmaxWarps = 4;
-constexpr int kMqaProducerWarps = 2;        // two key rows a thread
+constexpr int kMqaProducerWarps = 1;        // four key rows a lane (TMA gathers)
 constexpr int kMqaMmaWarp = 4;
-constexpr int kMqaThreads = (kMqaSoftmaxWarps + 1 + kMqaProducerWarps) * 32;   // 224
+constexpr int kMqaThreads = (kMqaSoftmaxWarps + 1 + kMqaProducerWarps) * 32;   // 192
 constexpr float kMqaLazyRescale = 8.f;   // log2 units: rescale O when the max grows by more
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -97,7 +99,8 @@ __device__ __forceinline__ void mqa_item(const MqaParams &p, int n, int &t, int 
 }
 
 __global__ void __launch_bounds__(kMqaThreads, 1)
-    sparse_mqa_kernel(const __grid_constant__ CUtensorMap tmap_q, const MqaParams p) {
+    sparse_mqa_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                      const __grid_constant__ CUtensorMap tmap_kv, const MqaParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -106,7 +109,7 @@ __global__ void __launch_bounds__(kMqaThreads, 1)
   uint8_t *sp = smem + MqaSmem::off_p;
   uint32_t *smask = reinterpret_cast<uint32_t *>(smem + MqaSmem::off_mask);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + MqaSmem::off_bar);
-  uint64_t *full = bars;                       // [stages] producer threads (64)
+  uint64_t *full = bars;                       // [stages] TMA bytes (lane 0 expects them)
   uint64_t *empty = full + kMqaStages;         // [stages] MMA commit after P V
   uint64_t *q_full = empty + kMqaStages;       // TMA bytes
   uint64_t *q_empty = q_full + 1;              // MMA commit after the item's last Q K^T
@@ -129,7 +132,7 @@ __global__ void __launch_bounds__(kMqaThreads, 1)
   }
   if (tid == 0) {
     for (int i = 0; i < kMqaStages; ++i) {
-      mbar_init(full + i, kMqaProducerWarps * 32);
+      mbar_init(full + i, 1);
       mbar_init(empty + i, 1);
     }
     mbar_init(q_full, 1);
@@ -144,6 +147,7 @@ __global__ void __launch_bounds__(kMqaThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmap_q);
+    tma_prefetch_desc(&tmap_kv);
   }
   if (warp > kMqaMmaWarp) {
     // head rows H..127 of the query tile stay zero (TMA fills rows 0..H-1)
@@ -162,13 +166,13 @@ __global__ void __launch_bounds__(kMqaThreads, 1)
   const int nitems = p.T * p.nsplit;
 
   if (warp > kMqaMmaWarp) {
-    // ---------------- producers: gather the selected kv rows ----------------
-    const int pt = tid - (kMqaMmaWarp + 1) * 32;       // key slots pt and pt + 64
-    const int pw = warp - (kMqaMmaWarp + 1);           // mask words pw and pw + 2
+    // ---------------- producer: gather the selected kv rows ----------------
+    const int pt = tid - (kMqaMmaWarp + 1) * 32;       // lane: tile rows 4pt .. 4pt+3
+    const int32_t oob_row = static_cast<int32_t>(static_cast<int64_t>(p.T / p.S_per_batch) * p.K);
     uint32_t g = 0, qn = 0;
-    int pending = -1;                                   // stage whose copies are not published
-    bool q_issued = false;
-    uint32_t q_phase = 0;
+    bool q_issued = false, k_issued = false;
+    uint32_t q_phase = 0, k_last_phase = 0;
+    uint32_t k_issued_mask = 0;
     bool ok = true;
     for (int n = blockIdx.x; n < nitems && ok; n += gridDim.x, ++qn) {
       int t, k0, k1, nt;
@@ -183,46 +187,45 @@ __global__ void __launch_bounds__(kMqaThreads, 1)
           q_phase = qn & 1u;
         }
       }
-      ok = __all_sync(0xffffffffu, ok) && !*abort_flag;
+      ok = __shfl_sync(0xffffffffu, ok, 0) && !*abort_flag;
       if (!ok) break;
-      const int64_t b = t / p.S_per_batch;
-      const uint16_t *kvb = p.kv + b * p.K * kMqaD;
+      const int64_t rb = static_cast<int64_t>(t / p.S_per_batch) * p.K;   // batch's first row
       const int *irow = p.idx + static_cast<int64_t>(t) * p.K_top;
       for (int j = 0; j < nt; ++j, ++g) {
         const uint32_t st = g % kMqaStages;
         if (!mbar_wait(empty + st, ((g / kMqaStages) & 1u) ^ 1u, ctl, 41)) { ok = false; break; }
-        uint8_t *dst = sk + st * MqaSmem::kTileBytes;
+        int32_t y[4];
+        uint32_t nib = 0;                               // validity of rows 4pt .. 4pt+3
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const int slot = pt + 64 * half;
-          const int key = k0 + j * kMqaTile + slot;
-          int row = -1;
-          if (key < k1) row = __ldg(irow + key);
+        for (int q = 0; q < 4; ++q) {
+          const int key = k0 + j * kMqaTile + 4 * pt + q;
+          const int row = key < k1 ? __ldg(irow + key) : -1;
           const bool valid = row >= 0 && row < p.K;
-          const uint32_t bal = __ballot_sync(0xffffffffu, valid);
-          if (lane == 0) smask[st * 4 + pw + 2 * half] = bal;
-          const uint16_t *src = kvb + (valid ? static_cast<int64_t>(row) : 0) * kMqaD;
+          y[q] = valid ? static_cast<int32_t>(rb + row) : oob_row;
+          nib |= static_cast<uint32_t>(valid) << q;
+        }
+        // validity words: slot 4l + q of the tile is bit (4l + q) % 32 of word l / 8
+        uint32_t word = nib << (4 * (pt & 7));
 #pragma unroll
-          for (int c = 0; c < 16; ++c)
-            cp_async16_zfill(dst + mqa_sw128(slot, c), src + c * 8, valid ? 16u : 0u);
-        }
-        cp_async_commit();
-        if (pending >= 0) {            // the previous tile: landed, visible to the MMA
-          cp_async_wait<1>();
-          fence_proxy_async_smem();
-          mbar_arrive(full + pending);
-        }
-        pending = static_cast<int>(st);
-      }
-      if (pending >= 0) {
-        cp_async_wait<0>();
-        fence_proxy_async_smem();
-        mbar_arrive(full + pending);
-        pending = -1;
+        for (int off = 1; off < 8; off <<= 1) word |= __shfl_xor_sync(0xffffffffu, word, off);
+        if ((pt & 7) == 0) smask[st * 4 + pt / 8] = word;
+        __syncwarp();
+        if (pt == 0) mbar_arrive_expect_tx(full + st, MqaSmem::kTileBytes);
+        __syncwarp();
+        uint8_t *dst = sk + st * MqaSmem::kTileBytes + 4 * pt * 128;
+        tma_gather4(dst, &tmap_kv, full + st, 0, y[0], y[1], y[2], y[3]);
+        tma_gather4(dst + 16384, &tmap_kv, full + st, 64, y[0], y[1], y[2], y[3]);
+        k_issued = true;
+        k_issued_mask |= 1u << st;
+        k_last_phase = (k_last_phase & ~(1u << st)) | (((g / kMqaStages) & 1u) << st);
       }
     }
-    cp_async_wait<0>();                 // nothing of ours in flight past this point
+    // every copy started here lands before the CTA can exit
     if (pt == 0 && q_issued) mbar_drain(q_full, q_phase, p.drain_limit_ns);
+    if (pt == 0 && k_issued)
+      for (int i = 0; i < kMqaStages; ++i)
+        if (k_issued_mask >> i & 1u) mbar_drain(full + i, k_last_phase >> i & 1u, p.drain_limit_ns);
+    __syncwarp();
   } else if (warp == kMqaMmaWarp) {
     // ---------------- MMA issuer ----------------
     const uint32_t idesc_s = idesc_bf16_f32(128, 128);

@@ -404,6 +404,8 @@ dsa_status_t launch_score(const dsa_indexer_desc_t *d, const void *q, const uint
   p.H = d->H;
   p.S = d->S;
   p.shared_cache = shared;
+  // a cache per token: each key tile is read by one token only
+  p.k_once = !causal && !shared;
   p.block_table = d->block_table;
   p.pages_per_seq = paged ? d->pages_per_seq : 0;
   p.num_pages = paged ? d->num_pages : 0;

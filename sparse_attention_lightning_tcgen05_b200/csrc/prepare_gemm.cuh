@@ -120,8 +120,9 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
                      const __grid_constant__ CUtensorMap tmap_b1,
                      const __grid_constant__ CUtensorMap tmap_b2, const PrepParams p) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned, by pointer arithmetic on the shared array, so that
+  // the compiler keeps every access through it in the shared address space
+  uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t *sa = smem + PrepSmem::off_a;
   uint8_t *sb = smem + PrepSmem::off_b;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + PrepSmem::off_bar);

@@ -75,6 +75,7 @@ struct ScoreParams {
   uint64_t wait_limit_ns;       // any single wait
   uint64_t drain_limit_ns;      // the drains on the way out (not the wait limit)
   int selftest_stall;           // the MMA warp first waits on a barrier nothing completes
+  int k_once;                   // every key tile is read by one query block only
 };
 
 __host__ __device__ constexpr int sf_atoms(int n_cols) { return (n_cols + 127) / 128; }
@@ -734,8 +735,9 @@ __global__ void __launch_bounds__((2 + kEPI + (kFP8 ? 1 : 0) + (kISS - 1)) * 32,
   constexpr int kGroups = kEPI / 4;
   constexpr int kAPS = kG;                       // accumulators per slot
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned, by pointer arithmetic on the shared array, so that
+  // the compiler keeps every access through it in the shared address space
+  uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const ScoreSmem L(kSTAGES, kQBUF, kNSUB, p.n_cols, kFP8, kEPI, kG);
   uint8_t *sk = smem + L.off_k;
   uint8_t *sq = smem + L.off_q;
@@ -833,6 +835,17 @@ __global__ void __launch_bounds__((2 + kEPI + (kFP8 ? 1 : 0) + (kISS - 1)) * 32,
       // row offset (no window padding: page boxes start on 4-word rows)
       const uint32_t tile_tx =
           L.k_stage_bytes + (kFP8 ? (p.block_table ? kBlockM * 4 : kSfBoxBytesK) : 0);
+      // keys read once (a cache per token) leave L2 first
+      const bool k_once = p.k_once != 0;
+      const uint64_t pol = l2_policy_evict_first();
+      auto load_k3 = [&](void *dst, int32_t c0, int32_t c1, int32_t c2) {
+        if (k_once) tma_load_3d_hint(dst, &tmap_k, full_k + st.idx, c0, c1, c2, pol);
+        else tma_load_3d(dst, &tmap_k, full_k + st.idx, c0, c1, c2);
+      };
+      auto load_ksf2 = [&](void *dst, int32_t c0, int32_t c1) {
+        if (k_once) tma_load_2d_hint(dst, &tmap_ksf, full_k + st.idx, c0, c1, pol);
+        else tma_load_2d(dst, &tmap_ksf, full_k + st.idx, c0, c1);
+      };
       bool need_q = true;
       while (c.left > 0) {
         const int g = cursor_tiles<kG>(c);
@@ -878,26 +891,23 @@ __global__ void __launch_bounds__((2 + kEPI + (kFP8 ? 1 : 0) + (kISS - 1)) * 32,
                   lp < p.pages_per_seq
                       ? __ldg(p.block_table + static_cast<int64_t>(c.q.z) * p.pages_per_seq + lp)
                       : p.num_pages;
-              tma_load_3d(dst + b * 128, &tmap_k, full_k + st.idx, 0, row, page);
+              load_k3(dst + b * 128, 0, row, page);
               if constexpr (kFP8) {
                 // boxes of >= 32 rows: at their row offset (a multiple of 128
                 // bytes); 16-row boxes: one 128-byte slot each
                 const int sf_off = box >= 32 ? 4 * b : 8 * b;
-                tma_load_2d(sksf + (st.idx * kG + i) * L.k_sf_bytes + sf_off, &tmap_ksf,
-                            full_k + st.idx, row, page);
+                load_ksf2(sksf + (st.idx * kG + i) * L.k_sf_bytes + sf_off, row, page);
               } else {
-                tma_load_3d(dst + kBlockM * 128 + b * 128, &tmap_k, full_k + st.idx, 64, row,
-                            page);
+                load_k3(dst + kBlockM * 128 + b * 128, 64, row, page);
               }
             }
             continue;
           }
-          tma_load_3d(dst, &tmap_k, full_k + st.idx, 0, y, c.q.z);
+          load_k3(dst, 0, y, c.q.z);
           if constexpr (kFP8) {
-            tma_load_2d(sksf + (st.idx * kG + i) * L.k_sf_bytes, &tmap_ksf, full_k + st.idx,
-                        y & ~(kSfPad - 1), c.q.z);
+            load_ksf2(sksf + (st.idx * kG + i) * L.k_sf_bytes, y & ~(kSfPad - 1), c.q.z);
           } else {
-            tma_load_3d(dst + kBlockM * 128, &tmap_k, full_k + st.idx, 64, y, c.q.z);
+            load_k3(dst + kBlockM * 128, 64, y, c.q.z);
           }
         }
         k_issued |= 1u << st.idx;

@@ -102,8 +102,9 @@ __global__ void __launch_bounds__(kMqaThreads, 1)
     sparse_mqa_kernel(const __grid_constant__ CUtensorMap tmap_q,
                       const __grid_constant__ CUtensorMap tmap_kv, const MqaParams p) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned, by pointer arithmetic on the shared array, so that
+  // the compiler keeps every access through it in the shared address space
+  uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t *sk = smem + MqaSmem::off_k;
   uint8_t *sq = smem + MqaSmem::off_q;
   uint8_t *sp = smem + MqaSmem::off_p;

@@ -122,11 +122,11 @@ def source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
-    """DRAM bytes per launch of the score kernel from the committed ncu
-    summary, or None when the summary is absent or the kernel source changed
-    since it was taken."""
-    path = os.path.join(ROOT, "profiles", f"score_kernel_{workload}.md")
+def profiled_traffic(workload: str, kernel: str = "score_kernel"):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu
+    summary (profiles/<kernel>_<workload>.md), or None when the summary is
+    absent or the kernel sources changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     if not os.path.exists(path):
         return None
     txt = open(path).read()
@@ -598,7 +598,8 @@ def run_mqa(args, wl):
     else:
         roof = {"bound": "hbm", "achieved": nbytes / (ms / 1e3) / 1e9, "peak": pk["hbm"],
                 "unit": "GB/s"}
-    roof.update(frac=roof["achieved"] / roof["peak"], traffic=None, kernel="sparse_mqa_kernel",
+    roof.update(frac=roof["achieved"] / roof["peak"],
+                traffic=profiled_traffic(wl.name, "sparse_mqa_kernel"), kernel="sparse_mqa_kernel",
                 roofline_ms=max(t_flops, t_bytes) * 1e3,
                 peak_source=f"{pk['src']} (MEASURED_PEAKS.json)")
     # the fp64 oracle on a bounded sample of tokens

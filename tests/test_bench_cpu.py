@@ -60,3 +60,54 @@ def test_workload_config_names_every_mode():
     assert "paged" in bench.workload_config(list(_cases())[-1])["caches"]
     for name in syn.WORKLOADS:
         assert name in bench.DEFAULTS
+
+
+def test_stratified_rows_cover_every_sequence_edge():
+    """The CPU baseline's row sample of a packed causal batch: the first and
+    last 16 rows of every sequence, seeded random rows, each row once, and
+    the valid pairs of those rows (row i of a sequence sees i + 1 keys)."""
+    wl = syn.Workload("c", syn.MODE_CAUSAL, T=5 + 40 + 100, H=4, D=128, index_topk=8,
+                      seqlens=(5, 40, 100), seed=0)
+    rows, pairs = bench.stratified_rows(wl, n_random=20)
+    assert rows == sorted(set(rows))
+    for a, L in ((0, 5), (5, 40), (45, 100)):
+        edge = set(range(a, a + min(L, 16))) | set(range(a + max(0, L - 16), a + L))
+        assert edge <= set(rows)
+    assert all(0 <= r < wl.T for r in rows)
+    P = oracle.Problem(wl, syn.generate(wl))
+    want = 0
+    for r in rows:
+        _, L, last, _ = P.row_info(r)
+        want += min(last + 1, L)
+    assert pairs == want
+
+
+def test_profiled_traffic_reads_only_a_current_summary(tmp_path, monkeypatch):
+    """The `traffic` of a bench line comes from profiles/<kernel>_<workload>.md
+    only when its src_hash is the sources' current hash."""
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    (tmp_path / "profiles").mkdir()
+    f = tmp_path / "profiles" / "score_kernel_w.md"
+    f.write_text("# x\n\nsrc_hash: `abc123`\ndram_bytes_per_launch: `12345`\n")
+    monkeypatch.setattr(bench, "source_hash", lambda: "abc123")
+    assert bench.profiled_traffic("w") == 12345.0
+    assert bench.profiled_traffic("missing") is None
+    monkeypatch.setattr(bench, "source_hash", lambda: "def456")
+    assert bench.profiled_traffic("w") is None
+    g = tmp_path / "profiles" / "sparse_mqa_kernel_m.md"
+    g.write_text("src_hash: `def456`\ndram_bytes_per_launch: `7`\n")
+    assert bench.profiled_traffic("m", "sparse_mqa_kernel") == 7.0
+
+
+def test_committed_profiles_name_their_sources_and_traffic():
+    """Every committed summary states the source hash it was taken on and
+    the DRAM bytes of one launch, in the form bench.py reads."""
+    import re
+    d = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "profiles")
+    names = [n for n in os.listdir(d) if n.endswith(".md")]
+    assert names
+    for n in names:
+        txt = open(os.path.join(d, n)).read()
+        assert re.search(r"src_hash:\s*`[0-9a-f]{16}`", txt), n
+        assert re.search(r"dram_bytes_per_launch:\s*`[0-9]+`", txt), n
+        assert "--clock-control none" in txt, n

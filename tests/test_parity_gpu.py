@@ -97,7 +97,7 @@ def test_decode_shared_cache_generic_heads(dsa):
     run_and_check(dsa, wl, syn.generate(wl))
 
 
-@pytest.mark.parametrize("H", [1, 4, 16, 64])
+@pytest.mark.parametrize("H", [1, 4, 16, 32, 64, 128])
 def test_causal_ragged_small(dsa, H):
     wl = causal_wl((1, 7, 127, 128, 129, 300, 1000), H=H, k=64, seed=H)
     run_and_check(dsa, wl, syn.generate(wl))
@@ -168,7 +168,7 @@ def test_fp8_integer_inputs_bit_exact(dsa, H):
     run_and_check(dsa, wl, syn.generate(wl, value_kind="int"), tol=TOL_FP8, exact=True)
 
 
-@pytest.mark.parametrize("H", [4, 64])
+@pytest.mark.parametrize("H", [4, 64, 128])
 def test_fp8_causal_ragged(dsa, H):
     wl = fp8_causal_wl((1, 127, 129, 300, 1000), H=H, k=64, seed=30 + H)
     run_and_check(dsa, wl, syn.generate(wl), tol=TOL_FP8)
@@ -204,7 +204,7 @@ def c4_wl(T, H, S, k, r=4, qs=0, dtype=syn.DTYPE_BF16, seed=0):
                         w_scale=1.0 / np.sqrt(H), seed=seed)
 
 
-@pytest.mark.parametrize("H", [4, 16, 64])
+@pytest.mark.parametrize("H", [4, 16, 64, 128])
 def test_compressed_small(dsa, H):
     """Rows that see no pooled slot, a few, and all of them; S ragged."""
     wl = c4_wl(T=300, H=H, S=70, k=24, r=4, qs=0, seed=50 + H)
